@@ -1,0 +1,298 @@
+"""Pins of the CPU fp64 oracle to things other than itself.
+
+Each test checks the oracle against a closed form, a library routine in a
+special case, a hand-derived worked example, an invariant the definition
+implies, or an independent brute force written here with plain loops.  The
+cases are chosen so that a plausible slip (a dropped ln c term, a sample
+instead of population std, statistics over the prefix, a flipped threshold
+comparison, a transposed operand, a lost max shift) fails at least one.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sol_attn_oracle as orc
+from block_sparse_attention_threshold_b200 import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _blocky(values, block, D=1):
+    """[len(values) * block, D] array whose block j rows all equal values[j]."""
+    return np.repeat(np.asarray(values, np.float64)[:, None], block, axis=0).repeat(D, axis=1)
+
+
+def _sdpa(q, k, v, scale, bias=None):
+    """torch's fp64 CPU scaled-dot-product attention for one head [N, D]."""
+    tq = torch.from_numpy(np.ascontiguousarray(q))[None, None]
+    tk = torch.from_numpy(np.ascontiguousarray(k))[None, None]
+    tv = torch.from_numpy(np.ascontiguousarray(v))[None, None]
+    mask = None if bias is None else torch.from_numpy(np.ascontiguousarray(bias))[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
+    return o[0, 0].numpy()
+
+
+def _tiny_inputs(rounded=True):
+    w = syn.workload("tiny_n1024")
+    if rounded:
+        q, k, v = (syn.bf16_bits_to_fp64(a) for a in syn.generate_bf16(w))
+    else:
+        q, k, v = syn.generate_fp64(w)
+    return w, q, k, v
+
+
+# ----------------------------------------------------------------------------- pooling
+
+def test_pool_constant_blocks_and_library_mean():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((64 * 5, 7))
+    means, counts = orc.pool_blocks(x, 64)
+    np.testing.assert_allclose(means, x.reshape(5, 64, 7).mean(axis=1), rtol=0, atol=1e-15)
+    assert list(counts) == [64] * 5
+    const = _blocky([1.5, -2.0, 0.25], 64, D=3)
+    m2, _ = orc.pool_blocks(const, 64)
+    assert np.array_equal(m2, np.array([[1.5] * 3, [-2.0] * 3, [0.25] * 3]))
+
+
+def test_pool_ragged_tail_counts():
+    x = np.arange(150 * 2, dtype=np.float64).reshape(150, 2)
+    means, counts = orc.pool_blocks(x, 64)
+    assert list(counts) == [64, 64, 22]
+    # brute force mean of the 22-row tail
+    tail = [sum(x[r, d] for r in range(128, 150)) / 22 for d in range(2)]
+    np.testing.assert_allclose(means[2], tail, rtol=1e-15)
+
+
+# ----------------------------------------------------------------------------- routing
+
+def _golden():
+    with open(os.path.join(GOLDEN, "route_worked_example.json")) as f:
+        return json.load(f)
+
+
+def _golden_head(g):
+    s = g["setup"]
+    block = s["block"]
+    k = _blocky(s["k_block_values"], block)
+    v = _blocky(s["v_block_values"], block)
+    q = np.ones_like(k)
+    return q, k, v, block, s["prefix_len"], s["scale"]
+
+
+def test_route_worked_example():
+    g = _golden()
+    e = g["expect"]
+    q, k, _, block, L, scale = _golden_head(g)
+    r = orc.route(q, k, block, L, 1.2, scale)
+    for i in range(1, 6):
+        assert r.mu[i] == pytest.approx(e["mu"], abs=1e-15)
+        assert r.sigma[i] == pytest.approx(e["sigma"], abs=1e-15)
+        assert r.thr[i] == pytest.approx(e["thr_tau_1.2"], abs=1e-14)
+        assert list(np.nonzero(r.keep[i, 1:])[0] + 1) == e["kept_video_tau_1.2"]
+        assert r.keep[i, 0]
+    assert r.keep[0].all()  # prefix query block dense
+    for tau, key in ((0.5, "kept_video_tau_0.5"), (-1.0, "kept_video_tau_-1")):
+        r = orc.route(q, k, block, L, tau, scale)
+        assert list(np.nonzero(r.keep[3, 1:])[0] + 1) == e[key]
+
+
+def test_route_tie_is_kept():
+    block = 64
+    k = _blocky([0.0, 2.0], block)
+    q = np.ones_like(k)
+    r = orc.route(q, k, block, 0, 1.0, 1.0)
+    assert r.thr[0] == 2.0
+    assert list(r.keep[0]) == [False, True]
+
+
+def test_worked_example_output_and_count_weight():
+    g = _golden()
+    q, k, v, block, L, scale = _golden_head(g)
+    out = orc.solattn_blocks(q, k, v, block, L, 1.2, scale, qblocks=[3])
+    assert np.allclose(out, g["expect"]["out_video_row_tau_1.2"], rtol=0, atol=g["expect"]["out_tol"])
+
+
+def test_route_special_taus_and_sigma_zero():
+    w, q, k, _ = _tiny_inputs()
+    for h in range(w.H):
+        r_all = orc.route(q[0, h], k[0, h], 64, w.prefix_len, -math.inf)
+        assert r_all.keep.all()
+        r_none = orc.route(q[0, h], k[0, h], 64, w.prefix_len, math.inf)
+        P = w.P
+        assert r_none.keep[:, :P].all() and r_none.keep[:P].all()
+        assert not r_none.keep[P:, P:].any()
+    # identical pooled keys -> sigma = 0 -> every block kept for any tau
+    kk = _blocky([0.7] * 8, 64, D=4)
+    qq = np.random.default_rng(2).standard_normal(kk.shape)
+    r = orc.route(qq, kk, 64, 64, 2.0)
+    assert (r.sigma[1:] == 0).all() and r.keep.all()
+
+
+def test_route_invariances():
+    w, q, k, _ = _tiny_inputs()
+    qh, kh = q[0, 0], k[0, 0]
+    base = orc.route(qh, kh, 64, w.prefix_len, 1.0)
+    # scaling queries by alpha > 0 leaves the mask unchanged
+    for alpha in (0.1, 3.0):
+        assert np.array_equal(orc.route(alpha * qh, kh, 64, w.prefix_len, 1.0).keep, base.keep)
+    # kept count is non-increasing in tau
+    counts = [orc.route(qh, kh, 64, w.prefix_len, t).keep.sum() for t in (-1, 0, 0.5, 1, 1.5, 2, 3)]
+    assert all(a >= b for a, b in zip(counts, counts[1:]))
+    # tau <= 0 keeps at least one video block per video query block (max >= mean)
+    r0 = orc.route(qh, kh, 64, w.prefix_len, 0.0)
+    assert r0.keep[w.P:, w.P:].any(axis=1).all()
+    # mean and std are those of numpy over the video scores
+    s = r0.score[w.P:, w.P:]
+    np.testing.assert_allclose(r0.mu[w.P:], s.mean(axis=1), rtol=1e-13)
+    np.testing.assert_allclose(r0.sigma[w.P:], s.std(axis=1, ddof=0), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def test_dense_rows_equal_library_sdpa():
+    w, q, k, v = _tiny_inputs(rounded=False)
+    scale = 1 / math.sqrt(w.D)
+    for h in range(w.H):
+        ref = _sdpa(q[0, h], k[0, h], v[0, h], scale)
+        np.testing.assert_allclose(orc.dense_rows(q[0, h], k[0, h], v[0, h]), ref, rtol=0, atol=1e-12)
+
+
+def test_tau_minus_inf_is_dense_attention():
+    for rounded in (False, True):
+        w, q, k, v = _tiny_inputs(rounded)
+        out = orc.solattn(q, k, v, 64, w.prefix_len, -math.inf)
+        for h in range(w.H):
+            ref = _sdpa(q[0, h], k[0, h], v[0, h], 1 / math.sqrt(w.D))
+            np.testing.assert_allclose(out[0, h], ref, rtol=0, atol=1e-12)
+
+
+def test_tau_plus_inf_is_attention_over_prefix_and_pooled_keys():
+    """tau = +inf: video rows attend to the prefix tokens plus one pooled key per
+    video block with additive bias ln 64 -- textbook attention with a float bias."""
+    w, q, k, v = _tiny_inputs()
+    L, P = w.prefix_len, w.P
+    scale = 1 / math.sqrt(w.D)
+    for h in range(w.H):
+        qh, kh, vh = q[0, h], k[0, h], v[0, h]
+        kbar = kh[L:].reshape(-1, 64, w.D).mean(axis=1)
+        vbar = vh[L:].reshape(-1, 64, w.D).mean(axis=1)
+        keys = np.concatenate([kh[:L], kbar])
+        vals = np.concatenate([vh[:L], vbar])
+        bias = np.concatenate([np.zeros(L), np.full(kbar.shape[0], math.log(64))])
+        ref = _sdpa(qh[L:], keys, vals, scale, np.broadcast_to(bias, (w.N - L, keys.shape[0])))
+        out = orc.solattn_blocks(qh, kh, vh, 64, L, math.inf, qblocks=range(P, w.M))
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+        # prefix query rows stay dense
+        out_p = orc.solattn_blocks(qh, kh, vh, 64, L, math.inf, qblocks=range(P))
+        np.testing.assert_allclose(out_p, _sdpa(qh[:L], kh, vh, scale), rtol=0, atol=1e-12)
+
+
+def test_identical_key_blocks_make_the_correction_exact():
+    """If every key and value of a block is the same vector, sum_t e^{q.k_t} v_t =
+    c e^{q.kbar} vbar, so Sol-Attn equals dense attention for every tau."""
+    rng = np.random.default_rng(7)
+    N, D, L = 64 * 10, 16, 128
+    kb = rng.standard_normal((N // 64, D))
+    vb = rng.standard_normal((N // 64, D))
+    k = np.repeat(kb, 64, axis=0)
+    v = np.repeat(vb, 64, axis=0)
+    q = rng.standard_normal((N, D)) * 2.0
+    ref = _sdpa(q, k, v, 1 / math.sqrt(D))
+    for tau in (-0.5, 0.0, 0.75, 1.5, math.inf):
+        r = orc.route(q, k, 64, L, tau)
+        if tau > 0:
+            assert not r.keep.all()  # some blocks really are skipped
+        out = orc.solattn_blocks(q, k, v, 64, L, tau)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_prefix_rows_are_dense_for_any_tau():
+    w, q, k, v = _tiny_inputs()
+    rows = range(w.prefix_len)
+    for tau in (0.0, 1.0, 2.0, math.inf):
+        out = orc.solattn(q, k, v, 64, w.prefix_len, tau, qblocks=range(w.P))
+        ref = orc.dense(q, k, v, rows=rows)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+def test_value_shift_invariance():
+    w, q, k, v = _tiny_inputs()
+    c = np.linspace(-1, 1, w.D)
+    a = orc.solattn(q, k, v, 64, w.prefix_len, 1.0)
+    b = orc.solattn(q, k, v + c, 64, w.prefix_len, 1.0)
+    np.testing.assert_allclose(b - a, np.broadcast_to(c, a.shape), rtol=0, atol=1e-12)
+
+
+def _brute_force_head(q, k, v, block, L, tau):
+    """Independent plain-loop Sol-Attn for tiny inputs (lists and math only)."""
+    N, D = len(q), len(q[0])
+    M, P = N // block, L // block
+    scale = 1.0 / math.sqrt(D)
+
+    def mean_block(x, j):
+        return [sum(x[t][d] for t in range(j * block, (j + 1) * block)) / block for d in range(D)]
+
+    def dot(a, b):
+        return sum(x * y for x, y in zip(a, b))
+
+    qb = [mean_block(q, j) for j in range(M)]
+    kb = [mean_block(k, j) for j in range(M)]
+    vb = [mean_block(v, j) for j in range(M)]
+    out = []
+    for i in range(M):
+        keep = [True] * M
+        if i >= P and M > P:
+            s = [scale * dot(qb[i], kb[j]) for j in range(P, M)]
+            mu = sum(s) / len(s)
+            sd = math.sqrt(sum((x - mu) ** 2 for x in s) / len(s))
+            if tau != -math.inf and sd != 0:
+                for j in range(P, M):
+                    keep[j] = s[j - P] >= mu + tau * sd
+        for r in range(i * block, (i + 1) * block):
+            terms = []  # (logit, value)
+            for j in range(M):
+                if keep[j]:
+                    for t in range(j * block, (j + 1) * block):
+                        terms.append((scale * dot(q[r], k[t]), v[t]))
+                else:
+                    terms.append((scale * dot(q[r], kb[j]) + math.log(block), vb[j]))
+            m = max(x for x, _ in terms)
+            den = sum(math.exp(x - m) for x, _ in terms)
+            out.append([sum(math.exp(x - m) * val[d] for x, val in terms) / den for d in range(D)])
+    return out
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.8, 1.5])
+def test_brute_force_tiny(tau):
+    rng = np.random.default_rng(11)
+    block, N, D, L = 8, 8 * 7, 3, 16
+    base = np.repeat(rng.standard_normal((N // block, D)), block, axis=0)
+    q = base + 0.5 * rng.standard_normal((N, D))
+    k = base + 0.5 * rng.standard_normal((N, D))
+    v = rng.standard_normal((N, D))
+    ref = np.array(_brute_force_head(q.tolist(), k.tolist(), v.tolist(), block, L, tau))
+    out = orc.solattn_blocks(q, k, v, block, L, tau)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    r = orc.route(q, k, block, L, tau)
+    assert r.keep.sum() < r.keep.size or tau == 0.0
+
+
+def test_dropping_the_count_weight_would_be_caught():
+    """Plant the mistake in a copy of the oracle's correction: the worked example flags it."""
+    g = _golden()
+    q, k, v, block, L, scale = _golden_head(g)
+    r = orc.route(q, k, block, L, 1.2, scale)
+    # Recompute the row with weight 1 instead of c_j for skipped blocks.
+    kept = np.nonzero(r.keep[3])[0]
+    skipped = np.nonzero(~r.keep[3])[0]
+    kv = np.array(g["setup"]["k_block_values"])
+    vv = np.array(g["setup"]["v_block_values"])
+    num = 64 * (np.exp(kv[kept]) * vv[kept]).sum() + (np.exp(kv[skipped]) * vv[skipped]).sum()
+    den = 64 * np.exp(kv[kept]).sum() + np.exp(kv[skipped]).sum()
+    wrong = num / den
+    assert abs(wrong - g["expect"]["out_video_row_tau_1.2"]) > 1e-3
