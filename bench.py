@@ -1,0 +1,442 @@
+"""Sol-Attn benchmark: dense-equivalent TFLOP/s of one forward over a workload.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--tau T]
+                [--impl reference]
+
+A step is one sol_attn_forward (block pooling + fused routing / attention /
+correction) over one batch of synthetic inputs resident in HBM.  The inputs
+(1 GB for the default refine workload) are larger than L2, so no flush is
+needed between steps.  Under torchrun each rank runs its own independent
+problem (weak scaling, no collective on the data path); the reported value is
+the dense-equivalent FLOPs of all ranks over the max-over-ranks time.
+
+`--impl reference` times the CPU fp64 oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Sol-Attn dense-equiv TFLOP/s & tensor-pipe % at N=16k-128k, τ=1.0-1.5"
+DEFAULT_WORKLOAD = "refine_n32768"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "block_sparse_attention_threshold_b200", "csrc")
+    for f in ("attn_kernel.cuh", "ptx.cuh"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+def oracle_sample_rate(w, tau, budget_s: float, rank_seed: int = 0):
+    """Dense-equivalent TFLOP/s of the CPU oracle on sampled query blocks.
+
+    Query blocks are drawn (seeded) across heads and evaluated one head batch
+    at a time in a thread pool until about `budget_s` of wall time is spent;
+    the rate is extrapolated from the blocks done.
+    """
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+
+    from block_sparse_attention_threshold_b200 import synthetic as syn
+    from oracle import sol_attn_oracle as orc
+
+    small = w.replace(H=min(w.H, 4))
+    qb, kb, vb = syn.generate_bf16(small)
+    cores = os.cpu_count() or 1
+    import contextlib
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limit = contextlib.nullcontext()
+    with limit:
+        return _oracle_rate(w, tau, budget_s, rank_seed, small, qb, kb, vb, cores)
+
+
+def _oracle_rate(w, tau, budget_s, rank_seed, small, qb, kb, vb, cores):
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+
+    from block_sparse_attention_threshold_b200 import synthetic as syn
+    from oracle import sol_attn_oracle as orc
+
+    heads = []
+    for h in range(small.H):
+        q64, k64, v64 = (syn.bf16_bits_to_fp64(a[0, h]) for a in (qb, kb, vb))
+        heads.append((q64, k64, v64, orc.route(q64, k64, 64, w.prefix_len, tau)))
+    rng = np.random.default_rng(1000 + rank_seed)
+    done = 0
+    t0 = time.perf_counter()
+
+    def one(job):
+        h, i = job
+        q64, k64, v64, r = heads[h]
+        orc.solattn_blocks(q64, k64, v64, 64, w.prefix_len, tau, qblocks=[i], routing=r)
+        return 1
+
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        while time.perf_counter() - t0 < budget_s:
+            jobs = [(int(rng.integers(small.H)), int(rng.integers(w.M))) for _ in range(cores)]
+            done += sum(ex.map(one, jobs))
+    dt = time.perf_counter() - t0
+    flops = done * 4.0 * 64 * w.N * w.D  # dense-equivalent work of the blocks done
+    return flops / dt / 1e12, cores, done, dt
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_threshold_b200 import abi, build, synthetic as syn
+
+    if rank == 0:
+        build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    abi.lib()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = syn.workload(args.workload)
+    if world > 1:
+        w = w.replace(seed=w.seed + 7919 * rank)  # an independent problem per rank
+    tau = args.tau if args.tau is not None else w.taus[0]
+    qb, kb, vb = syn.generate_bf16(w)
+    host = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (qb, kb, vb)]
+    q, k, v = (h.to(dev) for h in host)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    dense_flops = w.dense_flops()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def step():
+        abi.forward(q, k, v, tau, w.prefix_len, out=out, stream=stream)
+
+    # Counters (outside the timed region).
+    opts = abi.Opts()
+    cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+    opts.kept_pairs = cnt.data_ptr()
+    opts.exact_pairs = cnt.data_ptr() + 8
+    abi.forward(q, k, v, tau, w.prefix_len, out=out, opts=opts, stream=stream)
+    torch.cuda.synchronize()
+    st = abi.device_status()
+    if st != abi.OK:
+        raise RuntimeError(abi.status_string(st))
+    kept_pairs, exact_pairs = (int(x) for x in cnt.cpu().tolist())
+    total_pairs = w.B * w.H * w.M * w.M
+    skipped_pairs = total_pairs - kept_pairs
+    kept_flops = kept_pairs * 4.0 * 64 * 64 * w.D
+    corr_flops = skipped_pairs * 4.0 * 64 * w.D
+    exact_flops = exact_pairs * 4.0 * 64 * 64 * w.D
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = dense_flops * world / (ms * 1e-3) / 1e12
+
+    # Per-kernel timing for the roofline: pool and attend launched alone on
+    # the same stream, CUDA events around each launch.
+    nbytes, _ = abi.workspace_layout(w.B, w.H, w.N, w.D)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 5)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    pool_ms = timed(lambda: abi.pool(q, k, v, ws, stream=stream))
+    attend_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, stream=stream))
+    dense_ms = timed(lambda: abi.dense_forward(q, k, v, out=out, stream=stream))
+    peaks = measured_peaks()
+    pool_bytes = 3.0 * w.B * w.H * w.N * w.D * 2 + w.B * w.H * w.M * w.D * 12
+    achieved = (kept_flops + corr_flops) / (attend_ms * 1e-3) / 1e12
+    traffic = None
+    if os.path.exists(PROFILE_TRAFFIC):
+        with open(PROFILE_TRAFFIC) as f:
+            prof = json.load(f)
+        if prof.get("source_hash") == kernel_source_hash() and prof.get("workload") == w.name:
+            traffic = prof.get("dram_bytes_per_launch")
+
+    # End to end through the public call with host buffers: H2D of q, k, v
+    # from pinned memory, the forward, D2H of the output, every step.
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        for hsrc, dst in zip(host, (q, k, v)):
+            dst.copy_(hsrc, non_blocking=True)
+        abi.forward(q, k, v, tau, w.prefix_len, out=out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps)
+    e2e_value = dense_flops * world / (e2e_ms * 1e-3) / 1e12
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, cores, done, dt = oracle_sample_rate(w, tau, args.cpu_budget)
+            cpu = {"value": rate, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                   "sample": f"{done} query blocks of 64 rows (seeded, first 4 heads) of {w.name} "
+                             f"at tau={tau} in {dt:.1f} s, dense-equivalent FLOPs of those rows"}
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded video-grid Q/K/V, no model weights)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+                       "prefix_len": w.prefix_len, "tau": tau, "block": 64,
+                       "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2f} GB > L2 126 MB, no flush",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": traffic, "kernel": "sol_attn_fwd_kernel<128,false>",
+                         "peak_source": f"{peaks['source']} bf16 burst"},
+            "kernels": {
+                "attend_ms": attend_ms,
+                "pool_ms": pool_ms,
+                "pool_gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                "pool_hbm_frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "dense_ms": dense_ms,
+                "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+                "speedup_vs_dense": dense_ms / ms,
+                "kept_frac": kept_pairs / total_pairs,
+                "exact_frac": exact_pairs / total_pairs,
+                "actual_tflops_kept": kept_flops / (attend_ms * 1e-3) / 1e12,
+                "actual_tflops_kept_plus_corr": achieved,
+                "tensor_tflops_exact_union": exact_flops / (attend_ms * 1e-3) / 1e12,
+            },
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 3 * w.B * w.H * w.N * w.D * 2,
+                    "d2h_bytes_per_step": w.B * w.H * w.N * w.D * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+    return result
+
+
+def run_reference(args, rank):
+    from block_sparse_attention_threshold_b200 import synthetic as syn
+    if rank != 0:
+        return None
+    w = syn.workload(args.workload)
+    tau = args.tau if args.tau is not None else w.taus[0]
+    rates = []
+    t0 = time.perf_counter()
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, tau, max(1.0, args.ref_step_budget / 4))
+    for _ in range(args.steps):
+        r, cores, done, dt = oracle_sample_rate(w, tau, args.ref_step_budget)
+        rates.append(r)
+    value = statistics.mean(rates)
+    ms = 4.0 * w.N * w.N * w.D * w.B * w.H / (value * 1e12) * 1e3
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded video-grid Q/K/V, no model weights)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+                   "prefix_len": w.prefix_len, "tau": tau, "block": 64},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step ~{args.ref_step_budget:.0f} s of seeded query blocks "
+                                   f"(first 4 heads) of {w.name}; extrapolated dense-equivalent rate"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-step-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torchrun (one rank per GPU)")
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+"""ctypes binding of libsolattn.so (the C ABI in include/sol_attn.h).
+
+Argument marshalling only: tensors are passed as raw device pointers and the
+current CUDA stream as a handle.  Every step of the computation runs in the
+library's kernels; there is no fallback path.  If the library is missing the
+first call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsolattn.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_ARCH = 3
+ERR_CUDA = 4
+ERR_DEVICE_TIMEOUT = 5
+
+BLOCK = 64
+
+
+class SolAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class Opts(ctypes.Structure):
+    """Mirror of sol_attn_opts."""
+
+    _fields_ = [
+        ("kept_pairs", ctypes.c_void_p),
+        ("exact_pairs", ctypes.c_void_p),
+        ("debug_mask", ctypes.c_void_p),
+        ("softmax_scale", ctypes.c_float),
+        ("timeout_ms", ctypes.c_uint),
+        ("test_skip_first_k_load", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SIGS = {
+    "sol_attn_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sol_attn_forward_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
+    "sol_attn_dense_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sol_attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "sol_attn_pool": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sol_attn_attend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
+    "sol_attn_device_status": (_I, [_P]),
+    "sol_attn_status_string": (ctypes.c_char_p, [_I]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsolattn.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def declared_symbols(header: str) -> list:
+    """Function names declared in a C header (for export checks)."""
+    with open(header) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sol_attn_\w+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().sol_attn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise SolAttnError(status, where)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, D]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    return tuple(int(x) for x in q.shape)
+
+
+def _out_like(q, out):
+    import torch
+    if out is None:
+        return torch.empty_like(q)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    return out
+
+
+def forward(q, k, v, tau: float, prefix_len: int = 0, out=None, opts: Opts | None = None,
+            stream=None, block: int = BLOCK):
+    """Sol-Attn forward through sol_attn_forward_ex; returns `out`."""
+    B, H, N, D = _shape(q, k, v)
+    out = _out_like(q, out)
+    st = lib().sol_attn_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   B, H, N, D, block, float(tau), int(prefix_len),
+                                   ctypes.byref(opts) if opts is not None else None,
+                                   _stream(stream))
+    _check(st, "sol_attn_forward_ex")
+    return out
+
+
+def dense_forward(q, k, v, out=None, stream=None):
+    """Dense attention through sol_attn_dense_forward; returns `out`."""
+    B, H, N, D = _shape(q, k, v)
+    out = _out_like(q, out)
+    st = lib().sol_attn_dense_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      B, H, N, D, _stream(stream))
+    _check(st, "sol_attn_dense_forward")
+    return out
+
+
+def workspace_layout(B: int, H: int, N: int, D: int):
+    """(bytes, [4 section offsets]) of the pooled-summary workspace."""
+    offs = (ctypes.c_size_t * 4)()
+    n = lib().sol_attn_workspace_bytes(B, H, N, D, offs)
+    return int(n), [int(x) for x in offs]
+
+
+def pool(q, k, v, workspace, stream=None) -> None:
+    """Block means into `workspace` (a CUDA uint8 tensor) via sol_attn_pool."""
+    B, H, N, D = _shape(q, k, v)
+    st = lib().sol_attn_pool(q.data_ptr(), k.data_ptr(), v.data_ptr(), workspace.data_ptr(),
+                             B, H, N, D, _stream(stream))
+    _check(st, "sol_attn_pool")
+
+
+def attend(q, k, v, workspace, tau: float, prefix_len: int = 0, out=None,
+           opts: Opts | None = None, stream=None, block: int = BLOCK):
+    """Routing + attention on a pooled workspace via sol_attn_attend."""
+    B, H, N, D = _shape(q, k, v)
+    out = _out_like(q, out)
+    st = lib().sol_attn_attend(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               workspace.data_ptr(), B, H, N, D, block, float(tau),
+                               int(prefix_len), ctypes.byref(opts) if opts is not None else None,
+                               _stream(stream))
+    _check(st, "sol_attn_attend")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and read/clear the kernels' timeout word."""
+    return int(lib().sol_attn_device_status(_stream(stream)))
+
+
+def mask_words(M: int) -> int:
+    return (M + 31) // 32
+
+
+def unpack_mask(words, M: int):
+    """[..., ceil(M/32)] uint32 words (numpy) -> [..., M] bool."""
+    import numpy as np
+    w = np.ascontiguousarray(words).astype(np.uint32)
+    bits = ((w[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(bool)
+    return bits.reshape(*w.shape[:-1], -1)[..., :M]
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,331 @@
+// Host side of the C ABI declared in include/sol_attn.h: argument checks,
+// workspace, TMA descriptors and kernel launches.  No torch, no host syncs
+// (except sol_attn_device_status).
+#include "sol_attn.h"
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "attn_kernel.cuh"
+#include "pool_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCache {
+  std::once_flag once;
+  int status = SOL_ATTN_OK;  // SOL_ATTN_OK or SOL_ATTN_ERR_ARCH / _CUDA
+};
+DeviceCache g_dev[kMaxDevices];
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SOL_ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SOL_ATTN_ERR_UNSUPPORTED;
+  DeviceCache& c = g_dev[dev];
+  std::call_once(c.once, [&] {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      c.status = SOL_ATTN_ERR_CUDA;
+      return;
+    }
+    if (major != 10 || minor != 0) {
+      c.status = SOL_ATTN_ERR_ARCH;
+      return;
+    }
+    // Opt the attention kernels into their shared-memory footprint.
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<128, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sol::SmemPlan<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sol::SmemPlan<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<64, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sol::SmemPlan<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<64, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sol::SmemPlan<64>::kAlloc) == cudaSuccess;
+    c.status = ok ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+  });
+  return c.status;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D view [rows, D] of a bf16 array, 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Shape checks shared by every entry point.  Returns SOL_ATTN_OK, an error,
+// or -1 for an empty problem (nothing to do).
+int check_shape(int B, int H, int N, int D) {
+  if (B < 0 || H < 0 || N < 0) return SOL_ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SOL_ATTN_ERR_UNSUPPORTED;
+  if (N % SOL_ATTN_BLOCK != 0) return SOL_ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return -1;
+  if (N / SOL_ATTN_BLOCK > sol::kMaxBlocks) return SOL_ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N > INT_MAX) return SOL_ATTN_ERR_UNSUPPORTED;
+  return SOL_ATTN_OK;
+}
+
+int check_io(const void* q, const void* k, const void* v, const void* out) {
+  if (!q || !k || !v || !out) return SOL_ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return SOL_ATTN_ERR_INVALID_ARG;
+  return SOL_ATTN_OK;
+}
+
+int check_opts(const sol_attn_opts* o) {
+  if (o == nullptr) return SOL_ATTN_OK;
+  if (!(std::isfinite(o->softmax_scale)) || o->softmax_scale < 0.f) return SOL_ATTN_ERR_INVALID_ARG;
+  return SOL_ATTN_OK;
+}
+
+struct Workspace {
+  float* qbar;
+  float* kbar;
+  __nv_bfloat16* kbar_bf16;
+  __nv_bfloat16* vbar_bf16;
+};
+
+Workspace split_workspace(const void* ws, int B, int H, int N, int D) {
+  size_t off[4];
+  sol_attn_workspace_bytes(B, H, N, D, off);
+  auto* b = static_cast<uint8_t*>(const_cast<void*>(ws));
+  return Workspace{reinterpret_cast<float*>(b + off[0]), reinterpret_cast<float*>(b + off[1]),
+                   reinterpret_cast<__nv_bfloat16*>(b + off[2]),
+                   reinterpret_cast<__nv_bfloat16*>(b + off[3])};
+}
+
+int launch_pool(const void* q, const void* k, const void* v, const Workspace& w, int B, int H,
+                int N, int D, cudaStream_t s) {
+  const unsigned nblk = static_cast<unsigned>(static_cast<long long>(B) * H * (N / SOL_ATTN_BLOCK));
+  sol::PoolOut o{w.qbar, w.kbar, w.kbar_bf16, w.vbar_bf16};
+  dim3 grid(nblk, 3);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  if (D == 128)
+    sol::pool_kernel<128><<<grid, 128, 0, s>>>(qb, kb, vb, o);
+  else
+    sol::pool_kernel<64><<<grid, 128, 0, s>>>(qb, kb, vb, o);
+  return cudaGetLastError() == cudaSuccess ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+}
+
+int launch_attend(const void* q, const void* k, const void* v, void* out, const Workspace* w,
+                  int B, int H, int N, int D, float tau, int prefix_len, const sol_attn_opts* o,
+                  bool dense, cudaStream_t s) {
+  const int M = N / SOL_ATTN_BLOCK;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
+  const uint64_t prows = static_cast<uint64_t>(B) * H * M;
+  CUtensorMap mq, mk, mv, mkb, mvb;
+  if (!make_map(&mq, q, rows, D) || !make_map(&mk, k, rows, D) || !make_map(&mv, v, rows, D))
+    return SOL_ATTN_ERR_CUDA;
+  if (w != nullptr) {
+    if (!make_map(&mkb, w->kbar_bf16, prows, D) || !make_map(&mvb, w->vbar_bf16, prows, D))
+      return SOL_ATTN_ERR_CUDA;
+  } else {
+    mkb = mk;
+    mvb = mv;
+  }
+  sol::AttnParams p{};
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.M = M;
+  p.P = prefix_len / SOL_ATTN_BLOCK;
+  p.tiles_per_head = (M + 1) / 2;
+  p.tau = tau;
+  const float scale = (o != nullptr && o->softmax_scale > 0.f) ? o->softmax_scale
+                                                               : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.qbar = w ? w->qbar : nullptr;
+  p.kbar = w ? w->kbar : nullptr;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.debug_mask = o ? o->debug_mask : nullptr;
+  p.kept_pairs = o ? o->kept_pairs : nullptr;
+  p.exact_pairs = o ? o->exact_pairs : nullptr;
+  const unsigned tms = (o != nullptr && o->timeout_ms > 0) ? o->timeout_ms : 1000u;
+  p.timeout_ns = static_cast<uint64_t>(tms) * 1000000ull;
+  p.skip_first_k_arrival = o ? o->test_skip_first_k_load : 0;
+
+  const long long tiles = static_cast<long long>(B) * H * p.tiles_per_head;
+  dim3 grid(static_cast<unsigned>(tiles));
+  if (D == 128) {
+    const int smem = sol::SmemPlan<128>::kAlloc;
+    if (dense)
+      sol::sol_attn_fwd_kernel<128, true><<<grid, sol::kThreads, smem, s>>>(mq, mk, mv, mkb, mvb, p);
+    else
+      sol::sol_attn_fwd_kernel<128, false><<<grid, sol::kThreads, smem, s>>>(mq, mk, mv, mkb, mvb, p);
+  } else {
+    const int smem = sol::SmemPlan<64>::kAlloc;
+    if (dense)
+      sol::sol_attn_fwd_kernel<64, true><<<grid, sol::kThreads, smem, s>>>(mq, mk, mv, mkb, mvb, p);
+    else
+      sol::sol_attn_fwd_kernel<64, false><<<grid, sol::kThreads, smem, s>>>(mq, mk, mv, mkb, mvb, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+}
+
+int check_route_args(int block, float tau, int prefix_len, int N) {
+  if (block != SOL_ATTN_BLOCK) return SOL_ATTN_ERR_UNSUPPORTED;
+  if (std::isnan(tau)) return SOL_ATTN_ERR_INVALID_ARG;
+  if (prefix_len < 0 || prefix_len > N || prefix_len % SOL_ATTN_BLOCK != 0)
+    return SOL_ATTN_ERR_INVALID_ARG;
+  return SOL_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sol_attn_workspace_bytes(int B, int H, int N, int D, size_t* offsets) {
+  const int sc = check_shape(B, H, N, D);
+  if (sc != SOL_ATTN_OK) {
+    if (offsets) std::memset(offsets, 0, 4 * sizeof(size_t));
+    return 0;
+  }
+  const size_t rows = static_cast<size_t>(B) * H * (N / SOL_ATTN_BLOCK);
+  const size_t f32 = round256(rows * D * 4), b16 = round256(rows * D * 2);
+  if (offsets) {
+    offsets[0] = 0;
+    offsets[1] = f32;
+    offsets[2] = 2 * f32;
+    offsets[3] = 2 * f32 + b16;
+  }
+  return 2 * f32 + 2 * b16;
+}
+
+int sol_attn_pool(const void* q, const void* k, const void* v, void* workspace, int B, int H,
+                  int N, int D, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return SOL_ATTN_OK;
+  if (st != SOL_ATTN_OK) return st;
+  if (!q || !k || !v || !workspace || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  return launch_pool(q, k, v, split_workspace(workspace, B, H, N, D), B, H, N, D,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_attend(const void* q, const void* k, const void* v, void* out, const void* workspace,
+                    int B, int H, int N, int D, int block, float tau, int prefix_len,
+                    const sol_attn_opts* opts, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_opts(opts)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  const Workspace w = split_workspace(workspace, B, H, N, D);
+  return launch_attend(q, k, v, out, &w, B, H, N, D, tau, prefix_len, opts, false,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int B, int H,
+                        int N, int D, int block, float tau, int prefix_len,
+                        const sol_attn_opts* opts, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if ((st = check_opts(opts)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = sol_attn_workspace_bytes(B, H, N, D, nullptr);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return SOL_ATTN_ERR_CUDA;
+  const Workspace w = split_workspace(ws, B, H, N, D);
+  st = launch_pool(q, k, v, w, B, H, N, D, s);
+  if (st == SOL_ATTN_OK) st = launch_attend(q, k, v, out, &w, B, H, N, D, tau, prefix_len, opts, false, s);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == SOL_ATTN_OK) st = SOL_ATTN_ERR_CUDA;
+  return st;
+}
+
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                     int D, int block, float tau, int prefix_len, void* stream) {
+  return sol_attn_forward_ex(q, k, v, out, B, H, N, D, block, tau, prefix_len, nullptr, stream);
+}
+
+int sol_attn_dense_forward(const void* q, const void* k, const void* v, void* out, int B, int H,
+                           int N, int D, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return SOL_ATTN_OK;
+  if (st != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  return launch_attend(q, k, v, out, nullptr, B, H, N, D, -INFINITY, 0, nullptr, true,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SOL_ATTN_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, sol::g_sol_attn_error, sizeof(int)) != cudaSuccess)
+    return SOL_ATTN_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(sol::g_sol_attn_error, &zero, sizeof(int)) != cudaSuccess)
+      return SOL_ATTN_ERR_CUDA;
+    return SOL_ATTN_ERR_DEVICE_TIMEOUT;
+  }
+  return SOL_ATTN_OK;
+}
+
+const char* sol_attn_status_string(int status) {
+  switch (status) {
+    case SOL_ATTN_OK: return "SOL_ATTN_OK";
+    case SOL_ATTN_ERR_INVALID_ARG: return "SOL_ATTN_ERR_INVALID_ARG";
+    case SOL_ATTN_ERR_UNSUPPORTED: return "SOL_ATTN_ERR_UNSUPPORTED";
+    case SOL_ATTN_ERR_ARCH: return "SOL_ATTN_ERR_ARCH";
+    case SOL_ATTN_ERR_CUDA: return "SOL_ATTN_ERR_CUDA";
+    case SOL_ATTN_ERR_DEVICE_TIMEOUT: return "SOL_ATTN_ERR_DEVICE_TIMEOUT";
+    default: return "SOL_ATTN_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,150 @@
+/*
+ * sol_attn.h -- C ABI of the Sol-Attn library (libsolattn.so, sm_100a).
+ *
+ * Sol-Attn is training-free, query-adaptive block-sparse attention.  The
+ * pages that describe it give prose only; each entry point below names the
+ * passage it implements:
+ *
+ *  [R1] "NVIDIA 团队开源 Sol-H3 的 DGX Spark 版本" (arex-research 3d0ff631),
+ *       section "119.68 GiB memory pool", Sol-Attn bullet: blocks are picked
+ *       during attention; each query block filters light query-key scores
+ *       with its own threshold; selected blocks are exact; skipped blocks are
+ *       corrected from pooled K/V summaries; routing, sparse compute and
+ *       correction share one online softmax; no score map or routing index
+ *       tensor is written; the operator is compared with FA4 (dense).
+ *  [R2] Sol-H3 overview (yanziyuan 171844), "sparse attention" paragraph:
+ *       64-token blocks; "safety rail" paragraph: the packed
+ *       text | cond video | audio prefix always takes exact attention.
+ *  [R3] "MiniMax 官宣 NVIDIA Sol 团队 H3 加速" (arex-research 2a2a70ca),
+ *       section "speed-up comes from stacking every stage", Sol-Attn item:
+ *       keep threshold = mean + tau x std of the query block's scores.
+ *  [R4] "MiniMax 官推背书 Sol Engine" (arex-research 647c3193), section
+ *       "3.95x near-lossless": skipped blocks get a Taylor-approximation
+ *       compensation; this library implements its zeroth-order term
+ *       (count-weighted mean-key logit + ln c_j, mean value).
+ *
+ * Conventions shared by every entry point
+ *  - q, k, v, out: DEVICE pointers to contiguous bf16 arrays laid out
+ *    [B][H][N][D] (row-major, D fastest), 16-byte aligned, owned by the
+ *    caller.  out must not overlap q, k, v or the workspace.
+ *  - block must be 64; N and prefix_len must be multiples of 64; the
+ *    prefix is tokens [0, prefix_len) of every (b, h) sequence.
+ *  - D must be 64 or 128.  N / 64 must not exceed 4096 and B*H*N must fit
+ *    in a signed 32-bit integer (SOL_ATTN_ERR_UNSUPPORTED otherwise).
+ *  - B, H or N equal to 0 is an empty problem: SOL_ATTN_OK, nothing runs.
+ *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous with respect to the host and issues no host
+ *    synchronisation, except sol_attn_device_status().
+ *  - Arguments are validated before any work is enqueued; a call that
+ *    returns an error has enqueued nothing.  The library holds no state
+ *    besides per-device cached attributes and one device error word.
+ *  - Needs an sm_100 (B200-class) device: SOL_ATTN_ERR_ARCH otherwise.
+ */
+#ifndef SOL_ATTN_H
+#define SOL_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SOL_ATTN_BLOCK 64
+
+typedef enum {
+  SOL_ATTN_OK = 0,
+  SOL_ATTN_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment, prefix or tau */
+  SOL_ATTN_ERR_UNSUPPORTED = 2,     /* valid but outside what the kernels cover */
+  SOL_ATTN_ERR_ARCH = 3,            /* current device is not sm_100 */
+  SOL_ATTN_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+  SOL_ATTN_ERR_DEVICE_TIMEOUT = 5   /* a kernel wait gave up (see sol_attn_device_status) */
+} sol_attn_status;
+
+/* Optional extras of sol_attn_forward_ex / sol_attn_attend.  All pointers
+ * are DEVICE pointers and may be NULL.  Zero-initialise unused fields. */
+typedef struct {
+  /* += number of (query block, key block) pairs kept exact, forced prefix
+   * pairs included. */
+  unsigned long long* kept_pairs;
+  /* += number of (query block, key block) pairs the tensor cores computed
+   * exactly: each 128-row tile visits the union of its two query blocks'
+   * kept sets, so this is >= kept_pairs. */
+  unsigned long long* exact_pairs;
+  /* Keep bits for inspection, [B][H][M][ceil(M/32)] words, bit (j % 32) of
+   * word (j / 32) of row (b, h, i) set iff key block j is kept for query
+   * block i.  Only a debugging aid: when NULL (the normal case) no routing
+   * data leaves the chip. */
+  unsigned int* debug_mask;
+  /* Softmax (and score) scale; 0 means 1 / sqrt(D).  Must be finite, >= 0. */
+  float softmax_scale;
+  /* Limit of every in-kernel wait, in milliseconds; 0 means 1000. */
+  unsigned int timeout_ms;
+  /* Test hook, keep 0: the loader skips the first key tile of every CTA so
+   * the consumer's bounded wait runs out and the timeout path is exercised. */
+  int test_skip_first_k_load;
+} sol_attn_opts;
+
+/* Sol-Attn forward [R1]-[R4]: pooling, routing, exact attention on kept
+ * blocks, pooled correction of skipped blocks, one softmax.
+ *   tau: threshold multiplier; -INFINITY keeps every block (dense result),
+ *        +INFINITY keeps only the prefix; NaN is rejected.
+ *   prefix_len: tokens of exact prefix (prefix query rows are dense and
+ *        prefix key blocks are kept for every query block) [R2].
+ * Per query block i >= P = prefix_len/64: s_ij = scale * <mean q, mean k_j>
+ * over video key blocks j >= P; mu, sigma = population mean and std of
+ * those scores; keep j iff s_ij >= mu + tau * sigma (all kept when the
+ * scores are all equal).  A skipped block contributes logit
+ * scale * <q_r, mean k_j> + ln 64 and value mean v_j.
+ * Scratch: allocates sol_attn_workspace_bytes() with cudaMallocAsync on
+ * `stream` and frees it with cudaFreeAsync on the same stream. */
+int sol_attn_forward(const void* q, const void* k, const void* v, void* out, int B, int H,
+                     int N, int D, int block, float tau, int prefix_len, void* stream);
+
+/* Same as sol_attn_forward with the extras of `opts` (may be NULL). */
+int sol_attn_forward_ex(const void* q, const void* k, const void* v, void* out, int B, int H,
+                        int N, int D, int block, float tau, int prefix_len,
+                        const sol_attn_opts* opts, void* stream);
+
+/* Dense softmax attention softmax(q k^T / sqrt(D)) v: the comparator role of
+ * FA4 in [R1], and the tau = -INFINITY limit of Sol-Attn.  Same layout
+ * rules; needs no workspace and allocates nothing. */
+int sol_attn_dense_forward(const void* q, const void* k, const void* v, void* out, int B,
+                           int H, int N, int D, void* stream);
+
+/* Bytes of scratch sol_attn_pool / sol_attn_attend need, and (if `offsets`
+ * is not NULL) the byte offsets of its four sections, each 256-byte aligned,
+ * with BHM = B*H*N/64 rows of D values:
+ *   offsets[0] mean q   fp32 [BHM][D]
+ *   offsets[1] mean k   fp32 [BHM][D]
+ *   offsets[2] mean k   bf16 [BHM][D]  (round to nearest even of the fp32 mean)
+ *   offsets[3] mean v   bf16 [BHM][D]
+ * Returns 0 for invalid or empty shapes. */
+size_t sol_attn_workspace_bytes(int B, int H, int N, int D, size_t* offsets);
+
+/* Step 1 alone: block means of q, k, v [R1 "pooled K/V summaries", R2
+ * 64-token blocks] into `workspace` (device, caller-owned, at least
+ * sol_attn_workspace_bytes() bytes, 256-byte aligned). */
+int sol_attn_pool(const void* q, const void* k, const void* v, void* workspace, int B, int H,
+                  int N, int D, void* stream);
+
+/* Steps 2-6 alone (routing, exact + pooled attention, epilogue) on a
+ * workspace filled by sol_attn_pool for the same q, k, v.  `opts` may be
+ * NULL. */
+int sol_attn_attend(const void* q, const void* k, const void* v, void* out,
+                    const void* workspace, int B, int H, int N, int D, int block, float tau,
+                    int prefix_len, const sol_attn_opts* opts, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * kernels set when a bounded wait gives up.  SOL_ATTN_OK if none did,
+ * SOL_ATTN_ERR_DEVICE_TIMEOUT if one did, SOL_ATTN_ERR_CUDA if the
+ * synchronisation itself failed. */
+int sol_attn_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sol_attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_ATTN_H */

@@ -1,0 +1,131 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+and compare it with the CPU fp64 oracle on the same seeded inputs.
+
+Tolerances (the operator's acceptance bar):
+  * keep mask: >= 99.9 % of (query block, key block) pairs agree, and every
+    disagreement lies within 1e-3 * sigma_i of its threshold (fp32 routing on
+    the GPU vs fp64 in the oracle);
+  * output: relative L2 error <= 1e-2 and max abs error <= 2e-2 versus fp64
+    on the bf16 inputs.
+"""
+
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+from block_sparse_attention_threshold_b200 import abi, synthetic as syn
+from oracle import sol_attn_oracle as orc
+
+REL_L2 = 1e-2
+MAX_ABS = 2e-2
+MASK_AGREE = 0.999
+MASK_BAND = 1e-3
+
+
+def to_device(*arrays):
+    dev = torch.device("cuda", 0)
+    return [torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+            for a in arrays]
+
+
+def run_sol(w, tau, q, k, v, want_mask=True):
+    """Sol-Attn on device tensors; returns (out bf16 tensor, keep [B,H,M,M] bool or None,
+    kept_pairs, exact_pairs)."""
+    M = w.M
+    dev = q.device
+    opts = abi.Opts()
+    cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+    opts.kept_pairs = cnt.data_ptr()
+    opts.exact_pairs = cnt.data_ptr() + 8
+    mask = None
+    if want_mask:
+        mask = torch.zeros(w.B * w.H * M * abi.mask_words(M), dtype=torch.int32, device=dev)
+        opts.debug_mask = mask.data_ptr()
+    out = abi.forward(q, k, v, tau, w.prefix_len, opts=opts)
+    torch.cuda.synchronize()
+    status = abi.device_status()
+    assert status == abi.OK, abi.status_string(status)
+    keep = None
+    if want_mask:
+        words = mask.cpu().numpy().view(np.uint32).reshape(w.B, w.H, M, -1)
+        keep = abi.unpack_mask(words, M)
+    c = cnt.cpu().tolist()
+    return out, keep, int(c[0]), int(c[1])
+
+
+def _blas_single_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        import contextlib
+        return contextlib.nullcontext()
+
+
+def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False, workers=None):
+    """Compare GPU `out` (and `keep`) with the oracle, head by head in threads.
+
+    qblocks: query-block indices to check per head (None = all).
+    Returns a dict of metrics; raises AssertionError on a violated bound.
+    """
+    got_all = out.float().cpu().numpy()
+    B, H = w.B, w.H
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+
+    def one(bh):
+        b, h = bh
+        q64 = syn.bf16_bits_to_fp64(qb[b, h])
+        k64 = syn.bf16_bits_to_fp64(kb[b, h])
+        v64 = syn.bf16_bits_to_fp64(vb[b, h])
+        res = {}
+        blocks = range(w.M) if qblocks is None else qblocks
+        rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in blocks])
+        if dense:
+            ref = orc.dense_rows(q64, k64, v64, rows=rows)
+        else:
+            r = orc.route(q64, k64, 64, w.prefix_len, tau)
+            ref = orc.solattn_blocks(q64, k64, v64, 64, w.prefix_len, tau, qblocks=blocks, routing=r)
+            if keep is not None:
+                g = keep[b, h]
+                mism = g != r.keep
+                res["pairs"] = r.keep.size
+                res["mismatch"] = int(mism.sum())
+                if res["mismatch"]:
+                    ii, jj = np.nonzero(mism)
+                    dist = np.abs(r.score[ii, jj] - r.thr[ii]) / r.sigma[ii]
+                    res["worst_band"] = float(np.nanmax(dist))
+                res["kept"] = int(r.keep.sum())
+        got = got_all[b, h][rows].astype(np.float64)
+        res["err2"] = float(np.sum((got - ref) ** 2))
+        res["ref2"] = float(np.sum(ref ** 2))
+        res["maxabs"] = float(np.abs(got - ref).max())
+        return res
+
+    with _blas_single_thread():
+        with ThreadPoolExecutor(max_workers=workers or os.cpu_count()) as ex:
+            results = list(ex.map(one, jobs))
+    m = {
+        "rel_l2": math.sqrt(sum(r["err2"] for r in results) / sum(r["ref2"] for r in results)),
+        "max_abs": max(r["maxabs"] for r in results),
+    }
+    if keep is not None and not dense:
+        pairs = sum(r["pairs"] for r in results)
+        mism = sum(r["mismatch"] for r in results)
+        m["mask_agree"] = 1.0 - mism / pairs
+        m["mask_mismatch"] = mism
+        m["worst_band"] = max((r.get("worst_band", 0.0) for r in results), default=0.0)
+        m["oracle_kept"] = sum(r["kept"] for r in results)
+    return m
+
+
+def assert_parity(m):
+    assert m["rel_l2"] <= REL_L2, m
+    assert m["max_abs"] <= MAX_ABS, m
+    if "mask_agree" in m:
+        assert m["mask_agree"] >= MASK_AGREE, m
+        assert m["worst_band"] <= MASK_BAND, m
