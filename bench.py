@@ -170,6 +170,29 @@ def _oracle_rate(w, tau, budget_s, rank_seed, small, qb, kb, vb, cores):
     return flops / dt / 1e12, cores, done, dt
 
 
+# --------------------------------------------------------------------------- replicas
+
+def rank_workload(w, rank: int, world: int):
+    """Each rank runs its own independent problem: same shapes, its own seed."""
+    return w if world == 1 else w.replace(seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (the job ends with its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """All ranks' dense-equivalent FLOPs over the max-over-ranks step time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args, rank, world, local_rank):
@@ -186,9 +209,7 @@ def run_gpu(args, rank, world, local_rank):
     abi.lib()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = syn.workload(args.workload)
-    if world > 1:
-        w = w.replace(seed=w.seed + 7919 * rank)  # an independent problem per rank
+    w = rank_workload(syn.workload(args.workload), rank, world)
     tau = args.tau if args.tau is not None else w.taus[0]
     qb, kb, vb = syn.generate_bf16(w)
     host = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (qb, kb, vb)]
@@ -201,14 +222,6 @@ def run_gpu(args, rank, world, local_rank):
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     def step():
         abi.forward(q, k, v, tau, w.prefix_len, out=out, stream=stream)
@@ -245,8 +258,8 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    value = dense_flops * world / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    value = whole_job_tflops(dense_flops, world, ms)
 
     # Per-kernel timing for the roofline: pool and attend launched alone on
     # the same stream, CUDA events around each launch.
@@ -299,8 +312,8 @@ def run_gpu(args, rank, world, local_rank):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps)
-    e2e_value = dense_flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world, dev)
+    e2e_value = whole_job_tflops(dense_flops, world, e2e_ms)
 
     result = None
     if rank == 0:
