@@ -57,6 +57,7 @@ _SIGS = {
     "sol_attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "sol_attn_pool": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "sol_attn_attend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
+    "sol_attn_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sol_attn_device_status": (_I, [_P]),
     "sol_attn_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -134,6 +135,29 @@ def forward(q, k, v, tau: float, prefix_len: int = 0, out=None, opts: Opts | Non
                                    _stream(stream))
     _check(st, "sol_attn_forward_ex")
     return out
+
+
+def forward_noalloc(q, k, v, tau: float, prefix_len: int = 0, out=None, stream=None,
+                    block: int = BLOCK):
+    """Sol-Attn through sol_attn_forward_noalloc: the pooled workspace comes from
+    a fixed array inside the library, for callers that cannot allocate device
+    memory while they run.  Calls whose kernels overlap on the GPU race on that
+    array; the first call on a device must come before any stream capture."""
+    B, H, N, D = _shape(q, k, v)
+    out = _out_like(q, out)
+    st = lib().sol_attn_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        B, H, N, D, block, float(tau), int(prefix_len),
+                                        _stream(stream))
+    _check(st, "sol_attn_forward_noalloc")
+    return out
+
+
+def noalloc_max_workspace() -> int:
+    """SOL_ATTN_NOALLOC_MAX_WORKSPACE from the header: bytes of the fixed array."""
+    header = os.path.join(os.path.dirname(_HERE), "include", "sol_attn.h")
+    with open(header) as f:
+        m = re.search(r"#define\s+SOL_ATTN_NOALLOC_MAX_WORKSPACE\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    return int(m.group(1)) << int(m.group(2))
 
 
 def dense_forward(q, k, v, out=None, stream=None):

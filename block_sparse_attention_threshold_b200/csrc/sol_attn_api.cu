@@ -329,3 +329,77 @@ const char* sol_attn_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward.
+//
+// Some callers cannot call cudaMalloc while they run attention: a runtime
+// that reserves all device memory up front and forbids later allocation, an
+// inference server that must not let an allocator lock or fragment memory
+// between requests, or code running where the CUDA allocator may not be
+// entered.  sol_attn_forward_noalloc serves them.  It uses a fixed scratch
+// array compiled into this library instead of cudaMallocAsync, and it calls
+// no cudaMalloc, cudaFree or other allocating routine.
+//
+// The scratch array is a file-scope __device__ array of
+// SOL_ATTN_NOALLOC_MAX_WORKSPACE bytes.  Every GPU that loads the library
+// holds it until the process exits.  Host code cannot use the array's name
+// as a device address (on the host it names a stand-in), so the first call
+// on each device, with that device current, looks the address up with
+// cudaGetSymbolAddress and caches it.  Make that first call before any
+// stream capture.
+//
+// Every call shares the one array, so two calls whose kernels overlap on the
+// GPU (different streams, or different host threads) race on it.  Nothing
+// in it must start at zero: the pooling kernel writes every byte the
+// attention kernel reads, so the previous call's contents never leak into a
+// result.
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[SOL_ATTN_NOALLOC_MAX_WORKSPACE];
+
+struct NoAllocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  int status = SOL_ATTN_ERR_CUDA;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SOL_ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SOL_ATTN_ERR_UNSUPPORTED;
+  NoAllocScratch& s = g_noalloc[dev];
+  std::call_once(s.once, [&] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p != nullptr) {
+      s.ptr = p;
+      s.status = SOL_ATTN_OK;
+    }
+  });
+  *out = s.ptr;
+  return s.status;
+}
+
+}  // namespace
+
+extern "C" int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out,
+                                        int B, int H, int N, int D, int block, float tau,
+                                        int prefix_len, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if (sol_attn_workspace_bytes(B, H, N, D, nullptr) > SOL_ATTN_NOALLOC_MAX_WORKSPACE)
+    return SOL_ATTN_ERR_UNSUPPORTED;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  void* ws = nullptr;
+  if ((st = noalloc_scratch(&ws)) != SOL_ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Workspace w = split_workspace(ws, B, H, N, D);
+  st = launch_pool(q, k, v, w, B, H, N, D, s);
+  if (st == SOL_ATTN_OK)
+    st = launch_attend(q, k, v, out, &w, B, H, N, D, tau, prefix_len, nullptr, false, s);
+  return st;
+}

@@ -134,6 +134,32 @@ int sol_attn_attend(const void* q, const void* k, const void* v, void* out,
                     const void* workspace, int B, int H, int N, int D, int block, float tau,
                     int prefix_len, const sol_attn_opts* opts, void* stream);
 
+/* Largest workspace sol_attn_forward_noalloc can serve: 64 MiB, i.e.
+ * B*H*N <= 2,796,202 tokens at D = 128 (5,592,405 at D = 64). */
+#define SOL_ATTN_NOALLOC_MAX_WORKSPACE (64u << 20)
+
+/* Allocation-free variant of sol_attn_forward, for callers that cannot
+ * allocate device memory while they run (a runtime that reserves all memory
+ * up front, a server that must not enter the allocator between requests).
+ * The paper has no counterpart; this is a deployment convenience.
+ * Same arguments, layout and result as sol_attn_forward, but the pooled
+ * workspace is a fixed array compiled into the library
+ * (SOL_ATTN_NOALLOC_MAX_WORKSPACE bytes per device, held by every GPU that
+ * loads the library until the process exits).  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *  - Shapes whose sol_attn_workspace_bytes() exceed the array return
+ *    SOL_ATTN_ERR_UNSUPPORTED and enqueue nothing.
+ *  - The first call on each device (with that device current) looks up the
+ *    array's device address with cudaGetSymbolAddress.  Make that first
+ *    call before any stream capture.
+ *  - All calls share the one array.  Calls whose kernels overlap on the GPU
+ *    (other streams, other host threads) race on it and must be serialised
+ *    by the caller.  Nothing in it needs clearing: each call's pooling step
+ *    overwrites every byte that its attention step reads. */
+int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B,
+                             int H, int N, int D, int block, float tau, int prefix_len,
+                             void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * kernels set when a bounded wait gives up.  SOL_ATTN_OK if none did,
  * SOL_ATTN_ERR_DEVICE_TIMEOUT if one did, SOL_ATTN_ERR_CUDA if the
