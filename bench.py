@@ -170,6 +170,34 @@ def _oracle_rate(w, tau, budget_s, rank_seed, small, qb, kb, vb, cores):
     return flops / dt / 1e12, cores, done, dt
 
 
+# --------------------------------------------------------------------------- allocator
+
+def keep_pool_memory(device_index: int) -> bool:
+    """Let the device's default stream-ordered memory pool keep freed memory.
+
+    sol_attn_forward takes its scratch with cudaMallocAsync and returns it with
+    cudaFreeAsync.  With the pool's default release threshold (0) the memory
+    goes back to the driver at every synchronisation and the next call maps it
+    again, which costs milliseconds.  Keeping it is the usual setting for an
+    application that allocates every step; it lasts only for this process.
+    """
+    import ctypes
+    try:
+        cu = ctypes.CDLL("libcuda.so.1")
+        dev = ctypes.c_int()
+        pool = ctypes.c_void_p()
+        if cu.cuDeviceGet(ctypes.byref(dev), ctypes.c_int(device_index)) != 0:
+            return False
+        if cu.cuDeviceGetDefaultMemPool(ctypes.byref(pool), dev) != 0:
+            return False
+        threshold = ctypes.c_uint64(2 ** 64 - 1)
+        CU_MEMPOOL_ATTR_RELEASE_THRESHOLD = 4
+        return cu.cuMemPoolSetAttribute(pool, CU_MEMPOOL_ATTR_RELEASE_THRESHOLD,
+                                        ctypes.byref(threshold)) == 0
+    except OSError:
+        return False
+
+
 # --------------------------------------------------------------------------- replicas
 
 def rank_workload(w, rank: int, world: int):
@@ -209,6 +237,8 @@ def run_gpu(args, rank, world, local_rank):
     abi.lib()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    torch.zeros(1, device=dev)  # context up before touching the pool
+    pool_kept = keep_pool_memory(local_rank)
     w = rank_workload(syn.workload(args.workload), rank, world)
     tau = args.tau if args.tau is not None else w.taus[0]
     qb, kb, vb = syn.generate_bf16(w)
@@ -339,7 +369,8 @@ def run_gpu(args, rank, world, local_rank):
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
                        "prefix_len": w.prefix_len, "tau": tau, "block": 64,
                        "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2f} GB > L2 126 MB, no flush",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "mempool": "freed scratch kept by the pool" if pool_kept else "default pool"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                          "traffic": traffic, "kernel": "sol_attn_fwd_kernel<128,false>",

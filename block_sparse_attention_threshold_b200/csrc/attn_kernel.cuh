@@ -23,17 +23,22 @@
 //    blocks are always kept.
 //
 // Structure of one CTA (one 128-row query tile = query blocks 2t and 2t+1):
-//  warp 0     TMA producer: Q tile, then per stage a 128-key K tile and V tile
-//             (two kept 64-key blocks, possibly far apart, or 128 pooled keys);
-//  warp 1     tcgen05 issuer: S = Q K^T into TMEM, then O += P V with P read
-//             from TMEM (P overwrites S in place as bf16);
+//  warp 0     TMA producer: the Q tile, then per stage one 64-key block of K
+//             and one of V (a kept block, or 64 pooled keys for the
+//             correction) into separate 2-deep K and V rings, so the next K
+//             lands while the current block is still in the softmax;
+//  warp 1     tcgen05 issuer: S = Q K^T into one of two TMEM S buffers, so the
+//             next block's scores are computed while the softmax works on the
+//             current one; then O += P V with P read from TMEM (P overwrites
+//             its S buffer in place as bf16);
 //  warps 2-5  router (scores, mean/std, keep bits in shared memory), then
 //             online softmax (one TMEM lane = one query row), conditional O
 //             rescale, and the epilogue O / l -> bf16.
+// TMEM per CTA: S0 (64 columns) | S1 (64) | O (D) in 256 columns, so two
+// CTAs share an SM.
 // The tile visits the union of its two query blocks' kept sets; a row whose
 // block did not keep a visited key block masks it out and gets that block's
-// pooled correction instead.  Two CTAs share an SM (TMEM 2 x 256 columns),
-// so one CTA's softmax overlaps the other's MMAs.
+// pooled correction instead.
 #pragma once
 
 #include <cstdint>
@@ -43,13 +48,19 @@
 
 namespace sol {
 
-constexpr int kTileM = 128;     // query rows per CTA (two 64-token blocks)
-constexpr int kTileN = 128;     // keys per stage
+constexpr int kTileM = 128;       // query rows per CTA (two 64-token blocks)
+constexpr int kStageKeys = 64;    // keys per stage (one block)
+constexpr int kRingStages = 2;    // depth of the K ring and of the V ring
 constexpr int kMaxBlocks = 4096;  // largest M = N / 64 the router supports
 constexpr int kMaskWords = kMaxBlocks / 32;
 constexpr int kThreads = 192;
 constexpr float kLog2Block = 6.0f;        // log2(64): the ln c_j bias in log2 units
 constexpr float kRescaleSlack = 8.0f;     // keep a stale max while the new one is <= 2^8 larger
+#ifndef SOL_ATTN_FMA_EXP_PAIRS
+#define SOL_ATTN_FMA_EXP_PAIRS 2
+#endif
+// Of each 16 pairs of a 32-key half, this many take exp2 on the FMA pipe.
+constexpr int kFmaExpPairs = SOL_ATTN_FMA_EXP_PAIRS;
 
 // Device error word: 0 = fine, else the site of the first timed-out wait.
 __device__ int g_sol_attn_error = 0;
@@ -67,30 +78,45 @@ struct AttnParams {
   unsigned long long* kept_pairs;   // or null
   unsigned long long* exact_pairs;  // or null
   uint64_t timeout_ns;
-  int skip_first_k_arrival;  // test hook: producer never loads stage 0's K tile
+  int skip_first_k_arrival;  // test hook: producer never loads stage 0
 };
 
 template <int D>
 struct SmemPlan {
-  static constexpr int kTileBytes = kTileM * D * 2;  // 128 rows x D bf16
-  static constexpr int kChunkBytes = kTileM * 128;   // one 64-column chunk of a 128-row tile
+  static constexpr int kBlockBytes = kStageKeys * D * 2;  // one 64-key block of K (or V)
+  static constexpr int kChunkBytes = kStageKeys * 128;    // its 64-column chunk (8 KB)
+  static constexpr int kQChunkBytes = kTileM * 128;       // 64-column chunk of the Q tile
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kTileBytes;
-  static constexpr int kMaskA = kV + kTileBytes;
+  static constexpr int kK = kQ + kTileM * D * 2;           // K ring
+  static constexpr int kV = kK + kRingStages * kBlockBytes;  // V ring
+  static constexpr int kMaskA = kV + kRingStages * kBlockBytes;
   static constexpr int kMaskB = kMaskA + kMaskWords * 4;
   static constexpr int kMaskU = kMaskB + kMaskWords * 4;
   static constexpr int kQbar = kMaskU + kMaskWords * 4;  // 2 x D floats
   static constexpr int kRed = kQbar + 2 * D * 4;         // 32 floats
-  static constexpr int kBars = kRed + 32 * 4;            // 10 mbarriers
-  static constexpr int kMisc = kBars + 10 * 8;           // tmem base, abort flag
+  static constexpr int kBars = kRed + 32 * 4;
+  static constexpr int kNumBars = 4 * kRingStages + 2 + 6;
+  static constexpr int kMisc = kBars + kNumBars * 8;     // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;           // room to align the base to 1 KB
-  static_assert(2 * kMaxBlocks * 4 <= 2 * kTileBytes || D < 128, "score scratch must fit in K+V");
+  // The router's scores use the K and V rings before the first load.
+  static constexpr int kScores = kK;
+  static_assert(2 * kMaxBlocks * 4 <= 2 * kRingStages * kBlockBytes, "score scratch must fit in the rings");
 };
 
-enum BarId { kBarQ = 0, kBarKFull, kBarKEmpty, kBarVFull, kBarVEmpty, kBarSFull, kBarPFull,
-             kBarOFull, kBarDrain };
+// mbarriers: kfull[s], kempty[s], vfull[s], vempty[s], sfull[b], then singletons.
+enum BarId {
+  kBarKFull = 0,
+  kBarKEmpty = kRingStages,
+  kBarVFull = 2 * kRingStages,
+  kBarVEmpty = 3 * kRingStages,
+  kBarSFull = 4 * kRingStages,  // two S buffers
+  kBarQ = 4 * kRingStages + 2,
+  kBarPFull,
+  kBarOReady,
+  kBarOFull,
+  kBarDrain,
+};
 
 __device__ __forceinline__ bool mask_bit(const uint32_t* m, int j) {
   return (m[j >> 5] >> (j & 31)) & 1u;
@@ -108,14 +134,21 @@ __device__ __forceinline__ int next_bit(const uint32_t* m, int j, int nw) {
   return (w << 5) + __ffs(bits) - 1;
 }
 
-// One pass over the work of a tile.  Exact stages pair up the kept blocks of
-// the union mask in increasing order (j1 = -1 when the count is odd);
-// correction stages cover 128 pooled keys [128c, 128c + 128) that hold at
-// least one video block skipped by either query block.
+// Video key blocks of the 32-block mask word starting at block `lo`.
+__device__ __forceinline__ uint32_t video_bits(int lo, int M, int P) {
+  if (lo >= M || lo + 32 <= P) return 0u;
+  uint32_t v = lo < P ? (0xFFFFFFFFu << (P - lo)) : 0xFFFFFFFFu;
+  if (M - lo < 32) v &= (1u << (M - lo)) - 1u;
+  return v;
+}
+
+// The work of a tile, in order.  Exact stages: every block of the union of
+// the two query blocks' kept sets, ascending.  Correction stages: pooled
+// keys [64c, 64c + 64) holding at least one video block that either query
+// block skipped.
 struct Stage {
-  int j0, j1;     // exact: key blocks; correction: j0 = tile index c, j1 = -2
+  int j;      // exact: key block; correction: pooled tile c
   bool corr;
-  __device__ __forceinline__ int nkeys() const { return (corr || j1 >= 0) ? 128 : 64; }
 };
 
 struct StageIter {
@@ -126,33 +159,24 @@ struct StageIter {
     const int nw = (M + 31) >> 5;
     if (j < M) {
       const int j0 = next_bit(mU, j, nw);
-      if (j0 >= 0 && j0 < M) {
-        int j1 = next_bit(mU, j0 + 1, nw);
-        if (j1 >= M) j1 = -1;
-        s.j0 = j0;
-        s.j1 = j1;
+      if (j0 >= 0) {
+        s.j = j0;
         s.corr = false;
-        j = j1 < 0 ? M : j1 + 1;
+        j = j0 + 1;
         return true;
       }
       j = M;
     }
     if (dense) return false;
-    const int nc = (M + 127) >> 7;
+    const int nc = (M + 63) >> 6;
     while (c < nc) {
       const int cc = c++;
-      bool any = false;
-      for (int w = cc * 4; w < cc * 4 + 4 && w < nw; ++w) {
-        uint32_t video = 0xFFFFFFFFu;
-        const int lo = w * 32;
-        if (lo + 32 <= P) video = 0;
-        else if (lo < P) video = 0xFFFFFFFFu << (P - lo);
-        if (lo + 32 > M) video &= (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
-        if (((~mA[w]) | (~mB[w])) & video) { any = true; break; }
-      }
+      const int w0 = cc * 2;
+      uint32_t any = 0u;
+      for (int w = w0; w < w0 + 2 && w < nw; ++w)
+        any |= ((~mA[w]) | (~mB[w])) & video_bits(w * 32, M, P);
       if (any) {
-        s.j0 = cc;
-        s.j1 = -2;
+        s.j = cc;
         s.corr = true;
         return true;
       }
@@ -203,7 +227,7 @@ __device__ __forceinline__ void sm_reduce_minmax(float& mn_a, float& mx_a, float
 
 // Router: pooled scores of query blocks iA, iB against every video key
 // block, population mean/std, threshold, keep bits.  Runs on the 128
-// softmax threads; scores live in the (not yet used) K/V staging buffers.
+// softmax threads; scores live in the (not yet used) K/V rings.
 template <int D>
 __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, int iB, bool hasB,
                                            uint8_t* smem, int st) {
@@ -212,7 +236,7 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
   uint32_t* mB = reinterpret_cast<uint32_t*>(smem + L::kMaskB);
   float* sq = reinterpret_cast<float*>(smem + L::kQbar);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
-  float* sc = reinterpret_cast<float*>(smem + L::kK);  // [2][kMaxBlocks]
+  float* sc = reinterpret_cast<float*>(smem + L::kScores);  // [2][kMaxBlocks]
   const int M = p.M, P = p.P, nv = M - P;
   const int nw = (M + 31) >> 5;
   const bool videoA = iA >= P, videoB = hasB && iB >= P;
@@ -225,23 +249,66 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
       sq[D + d] = qb[d];
     }
     named_bar_sync(1, 128);
-    // One thread per video key block: 16-byte loads of its pooled key row.
-    const float* kb = p.kbar + static_cast<size_t>(bh) * M * D;
-    for (int j = P + st; j < M; j += 128) {
-      const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-      float da = 0.f, db = 0.f;
-#pragma unroll 8
-      for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 kv = __ldg(row + d4);
-        const float4 a = reinterpret_cast<const float4*>(sq)[d4];
-        const float4 b = reinterpret_cast<const float4*>(sq + D)[d4];
-        da = fmaf(a.x, kv.x, da); da = fmaf(a.y, kv.y, da);
-        da = fmaf(a.z, kv.z, da); da = fmaf(a.w, kv.w, da);
-        db = fmaf(b.x, kv.x, db); db = fmaf(b.y, kv.y, db);
-        db = fmaf(b.z, kv.z, db); db = fmaf(b.w, kv.w, db);
+    // Scores, 32 key blocks per warp step: lane l holds dims [D/32 * l, +D/32)
+    // of every row, so each row is one coalesced load of the warp; the 32
+    // partial dot products per lane are then reduced across lanes by a
+    // butterfly that leaves row (base + l)'s score in lane l.
+    {
+      constexpr int kDpl = D / 32;  // dims per lane: 4 (D = 128) or 2 (D = 64)
+      const int lane = st & 31, wq = st >> 5;
+      float qa[kDpl], qb[kDpl];
+#pragma unroll
+      for (int d = 0; d < kDpl; ++d) {
+        qa[d] = sq[lane * kDpl + d];
+        qb[d] = sq[D + lane * kDpl + d];
       }
-      sc[j - P] = da * p.scale;
-      sc[kMaxBlocks + j - P] = db * p.scale;
+      const float* kb = p.kbar + static_cast<size_t>(bh) * M * D + lane * kDpl;
+      for (int base = P + wq * 32; base < M; base += 128) {
+        float pa[32], pb[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+          const int j = base + rr;
+          float kv[kDpl];
+          if (j < M) {
+            if constexpr (kDpl == 4) {
+              const float4 x = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D));
+              kv[0] = x.x; kv[1] = x.y; kv[2] = x.z; kv[3] = x.w;
+            } else {
+              const float2 x = __ldg(reinterpret_cast<const float2*>(kb + static_cast<size_t>(j) * D));
+              kv[0] = x.x; kv[1] = x.y;
+            }
+          } else {
+#pragma unroll
+            for (int d = 0; d < kDpl; ++d) kv[d] = 0.f;
+          }
+          float da = 0.f, db = 0.f;
+#pragma unroll
+          for (int d = 0; d < kDpl; ++d) {
+            da = fmaf(qa[d], kv[d], da);
+            db = fmaf(qb[d], kv[d], db);
+          }
+          pa[rr] = da;
+          pb[rr] = db;
+        }
+#pragma unroll
+        for (int lvl = 16; lvl >= 1; lvl >>= 1) {
+          const bool upper = (lane & lvl) != 0;
+#pragma unroll
+          for (int i = 0; i < lvl; ++i) {
+            const float sa = upper ? pa[i] : pa[i + lvl];
+            const float ka = upper ? pa[i + lvl] : pa[i];
+            const float sb = upper ? pb[i] : pb[i + lvl];
+            const float kb2 = upper ? pb[i + lvl] : pb[i];
+            pa[i] = ka + __shfl_xor_sync(0xFFFFFFFFu, sa, lvl);
+            pb[i] = kb2 + __shfl_xor_sync(0xFFFFFFFFu, sb, lvl);
+          }
+        }
+        const int j = base + lane;
+        if (j < M) {
+          sc[j - P] = pa[0] * p.scale;
+          sc[kMaxBlocks + j - P] = pb[0] * p.scale;
+        }
+      }
     }
     named_bar_sync(1, 128);
     // Pass 1: mean (and exact-equality check through min/max).
@@ -310,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   using L = SmemPlan<D>;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kTmemCols = 256;
-  constexpr uint32_t kColS = 0, kColO = 128;
+  constexpr uint32_t kColO = 128;  // S buffer b at columns [64 b, 64 b + 64)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -336,13 +403,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   int* err = &g_sol_attn_error;
 
   if (tid == 0) {
+    for (int i = 0; i < kRingStages; ++i) {
+      mbar_init(&bars[kBarKFull + i], 1);
+      mbar_init(&bars[kBarKEmpty + i], 1);
+      mbar_init(&bars[kBarVFull + i], 1);
+      mbar_init(&bars[kBarVEmpty + i], 1);
+    }
+    mbar_init(&bars[kBarSFull + 0], 1);
+    mbar_init(&bars[kBarSFull + 1], 1);
     mbar_init(&bars[kBarQ], 1);
-    mbar_init(&bars[kBarKFull], 1);
-    mbar_init(&bars[kBarKEmpty], 1);
-    mbar_init(&bars[kBarVFull], 1);
-    mbar_init(&bars[kBarVEmpty], 1);
-    mbar_init(&bars[kBarSFull], 1);
     mbar_init(&bars[kBarPFull], 128);
+    mbar_init(&bars[kBarOReady], 1);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarDrain], 1);
     *abort_flag = 0;
@@ -358,29 +429,28 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = *tmem_holder;
 
   // Q tile first: it does not depend on the routing.
-  const size_t row0 = static_cast<size_t>(bh) * p.N + static_cast<size_t>(qt) * kTileM;
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    const size_t row0 = static_cast<size_t>(bh) * p.N + static_cast<size_t>(qt) * kTileM;
     mbar_arrive_expect_tx(&bars[kBarQ], kTileM * D * 2);
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int c = 0; c < kChunks; ++c)
-        tma_load_2d(sQ + c * L::kChunkBytes + h * 64 * 128, &tmQ, &bars[kBarQ], c * 64,
+        tma_load_2d(sQ + c * L::kQChunkBytes + h * 64 * 128, &tmQ, &bars[kBarQ], c * 64,
                     static_cast<int>(row0 + h * 64));
   }
 
-  // Routing (softmax warps), or the all-kept mask of the dense kernel.
   if (warp >= 2) {
     const int st = tid - 64;
     if (kDense) {
       for (int w = st; w < nw; w += 128) {
         const int lo = w * 32;
-        const uint32_t full = (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
-        mA[w] = full;
-        mB[w] = full;
+        const uint32_t fullw = (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
+        mA[w] = fullw;
+        mB[w] = fullw;
       }
     } else {
       route_tile<D>(p, bh, iA, iB, hasB, smem, st);
@@ -400,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (p.kept_pairs != nullptr && kept) atomicAdd(p.kept_pairs, kept);
       if (p.exact_pairs != nullptr && uni) atomicAdd(p.exact_pairs, uni);
     }
-    fence_proxy_async_smem();  // scores were written to K/V staging by generic stores
+    fence_proxy_async_smem();  // scores were written to the rings by generic stores
   }
   __syncthreads();
 
@@ -414,153 +484,250 @@ __global__ void __launch_bounds__(kThreads, 2)
       int n = 0;
       bool ok = true;
       while (ok && it.next(s, mU, mA, mB, M, P, kDense)) {
-        const int nhalves = s.corr ? 2 : (s.j1 >= 0 ? 2 : 1);
-        const uint32_t bytes = nhalves * kChunks * 64 * 128;
-        const CUtensorMap* mk = s.corr ? &tmKb : &tmK;
-        const CUtensorMap* mv = s.corr ? &tmVb : &tmV;
-        int r[2];
-        if (s.corr) {
-          r[0] = static_cast<int>(prow_head + s.j0 * 128);
-          r[1] = r[0] + 64;
-        } else {
-          r[0] = static_cast<int>(krow_head + static_cast<size_t>(s.j0) * 64);
-          r[1] = static_cast<int>(krow_head + static_cast<size_t>(s.j1 < 0 ? 0 : s.j1) * 64);
-        }
-        if (n > 0) ok = mbar_wait(&bars[kBarKEmpty], (n - 1) & 1, abort_flag, err, 1, p.timeout_ns);
+        const int slot = n % kRingStages;
+        const uint32_t use_parity = ((n / kRingStages) - 1) & 1;
+        const int row = static_cast<int>(s.corr ? prow_head + static_cast<size_t>(s.j) * 64
+                                                : krow_head + static_cast<size_t>(s.j) * 64);
+        if (n >= kRingStages)
+          ok = mbar_wait(&bars[kBarKEmpty + slot], use_parity, abort_flag, err, 1, p.timeout_ns);
         if (!ok) break;
         if (!(p.skip_first_k_arrival && n == 0)) {
-          mbar_arrive_expect_tx(&bars[kBarKFull], bytes);
-          for (int h = 0; h < nhalves; ++h)
-            for (int c = 0; c < kChunks; ++c)
-              tma_load_2d(sK + c * L::kChunkBytes + h * 64 * 128, mk, &bars[kBarKFull], c * 64, r[h]);
-        }
-        if (n > 0) ok = mbar_wait(&bars[kBarVEmpty], (n - 1) & 1, abort_flag, err, 2, p.timeout_ns);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bars[kBarVFull], bytes);
-        for (int h = 0; h < nhalves; ++h)
+          mbar_arrive_expect_tx(&bars[kBarKFull + slot], L::kBlockBytes);
+#pragma unroll
           for (int c = 0; c < kChunks; ++c)
-            tma_load_2d(sV + c * L::kChunkBytes + h * 64 * 128, mv, &bars[kBarVFull], c * 64, r[h]);
+            tma_load_2d(sK + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmKb : &tmK,
+                        &bars[kBarKFull + slot], c * 64, row);
+        }
+        if (n >= kRingStages)
+          ok = mbar_wait(&bars[kBarVEmpty + slot], use_parity, abort_flag, err, 2, p.timeout_ns);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars[kBarVFull + slot], L::kBlockBytes);
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_2d(sV + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmVb : &tmV,
+                      &bars[kBarVFull + slot], c * 64, row);
         ++n;
       }
       if (!ok || *abort_flag) {
         // Let loads already issued land before the CTA's shared memory is released.
         const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 2000000ull) { }
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kStageKeys, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
+      int total = 0;
+      {
+        StageIter it;
+        Stage s;
+        while (it.next(s, mU, mA, mB, M, P, kDense)) ++total;
+      }
       bool ok = mbar_wait(&bars[kBarQ], 0, abort_flag, err, 3, p.timeout_ns);
-      StageIter it;
-      Stage s;
-      int n = 0;
-      while (ok && it.next(s, mU, mA, mB, M, P, kDense)) {
-        const int nk = s.nkeys();
-        ok = mbar_wait(&bars[kBarKFull], n & 1, abort_flag, err, 4, p.timeout_ns);
-        if (!ok) break;
+      // S(n) = Q K(n)^T into S buffer n % 2; A = Q (K-major SW128), B = K.
+      auto issue_s = [&](int n) -> bool {
+        const int slot = n % kRingStages;
+        if (!mbar_wait(&bars[kBarKFull + slot], (n / kRingStages) & 1, abort_flag, err, 4, p.timeout_ns))
+          return false;
         tc_fence_after();
-        const uint32_t idesc_qk = idesc_bf16_f32(kTileM, nk, false);
+        const uint32_t ka = sKa + slot * L::kBlockBytes;
+        const uint32_t dcol = tmem + 64u * (n & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColS, sdesc_sw128(sQa + off, 16, 1024), sdesc_sw128(sKa + off, 16, 1024),
+          const uint32_t qoff = (kk >> 2) * L::kQChunkBytes + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+          mma_bf16_ss(dcol, sdesc_sw128(sQa + qoff, 16, 1024), sdesc_sw128(ka + koff, 16, 1024),
                       idesc_qk, kk > 0);
         }
-        mma_commit(&bars[kBarSFull]);
-        mma_commit(&bars[kBarKEmpty]);
+        mma_commit(&bars[kBarSFull + (n & 1)]);
+        mma_commit(&bars[kBarKEmpty + slot]);
+        return true;
+      };
+      if (ok && total > 0) ok = issue_s(0);
+      if (ok && total > 1) ok = issue_s(1);
+      for (int n = 0; ok && n < total; ++n) {
+        const int slot = n % kRingStages;
         ok = mbar_wait(&bars[kBarPFull], n & 1, abort_flag, err, 5, p.timeout_ns);
-        if (ok) ok = mbar_wait(&bars[kBarVFull], n & 1, abort_flag, err, 6, p.timeout_ns);
+        if (ok) ok = mbar_wait(&bars[kBarVFull + slot], (n / kRingStages) & 1, abort_flag, err, 6, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        for (int kk = 0; kk < nk / 16; ++kk) {
-          mma_bf16_ts(tmem + kColO, tmem + kColS + kk * 8,
-                      sdesc_sw128(sVa + kk * 16 * 128, L::kChunkBytes, 1024), idesc_pv,
-                      (n > 0 || kk > 0) ? 1u : 0u);
+        // O += P V: A = P from S buffer n % 2 (TMEM), B = V (MN-major).
+        const uint32_t pcol = tmem + 64u * (n & 1);
+        const uint32_t va = sVa + slot * L::kBlockBytes;
+#pragma unroll
+        for (int kk = 0; kk < kStageKeys / 16; ++kk) {
+          mma_bf16_ts(tmem + kColO, pcol + kk * 8, sdesc_sw128(va + kk * 16 * 128, L::kChunkBytes, 1024),
+                      idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bars[kBarVEmpty]);
-        ++n;
+        mma_commit(&bars[kBarVEmpty + slot]);
+        mma_commit(&bars[kBarOReady]);
+        // The next S into this buffer runs after this PV (tcgen05.mma from one
+        // thread executes in issue order), so P is read before it is overwritten.
+        if (n + 2 < total) ok = issue_s(n + 2);
       }
       mma_commit(&bars[kBarOFull]);
       mma_commit(&bars[kBarDrain]);
       // Drain: the CTA must not free TMEM while MMAs are still running.
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(&bars[kBarDrain], 0) && global_timer_ns() - t0 < 2000000000ull) { }
+      while (!mbar_try_wait_sleep(&bars[kBarDrain], 0, kWaitHintNs) &&
+             global_timer_ns() - t0 < 2000000000ull) {
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int sp = warp & 3;               // TMEM sub-partition of this warp
-    const int r = sp * 32 + lane;          // query row within the tile
+    const int sp = warp & 3;
+    const int r = sp * 32 + lane;
     const uint32_t* rowmask = r < 64 ? mA : mB;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sp * 32) << 16);
+    const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
     float m = -INFINITY, l = 0.f;
     StageIter it;
     Stage s;
     int n = 0;
     bool ok = true;
     while (it.next(s, mU, mA, mB, M, P, kDense)) {
-      ok = mbar_wait(&bars[kBarSFull], n & 1, abort_flag, err, 7, p.timeout_ns);
+      const uint32_t scol = lane_addr + 64u * (n & 1);
+      ok = mbar_wait(&bars[kBarSFull + (n & 1)], (n >> 1) & 1, abort_flag, err, 7, p.timeout_ns);
       if (!ok) break;
       tc_fence_after();
-      const int nch = s.nkeys() / 32;  // 32-key chunks in this stage (2 or 4)
-      // S row -> registers (all of it before P overwrites it in place).
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
-        if (ch < nch) tmem_ld32(lane_addr + kColS + ch * 32, sv[ch]);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
-        if (ch < nch) tmem_ld_wait(sv[ch]);
-      // Scaled, masked logits in log2 units, written back over sv.
-      float tmax = -INFINITY;
+      // Which of the 64 columns this row uses (warp-uniform: one query block per warp).
+      uint32_t use0, use1;
       if (!s.corr) {
-        const bool k0 = mask_bit(rowmask, s.j0);
-        const bool k1 = s.j1 >= 0 && mask_bit(rowmask, s.j1);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          if (ch < nch) {
-            const bool keep = ch < 2 ? k0 : k1;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float xv = keep ? __uint_as_float(sv[ch][c]) * p.scale_log2 : -INFINITY;
-              sv[ch][c] = __float_as_uint(xv);
-              tmax = fmaxf(tmax, xv);
-            }
-          }
-        }
+        use0 = use1 = mask_bit(rowmask, s.j) ? 0xFFFFFFFFu : 0u;
       } else {
-        const int jb = s.j0 * 128;
+        const int lo = s.j * 64;
+        const uint32_t v0 = video_bits(lo, M, P), v1 = video_bits(lo + 32, M, P);
+        use0 = v0 ? (~rowmask[lo >> 5] & v0) : 0u;
+        use1 = v1 ? (~rowmask[(lo >> 5) + 1] & v1) : 0u;
+      }
+      uint32_t pk0[16], pk1[16];
+      float alpha = 1.0f;
+      bool warp_need = false;
+      if (__any_sync(0xFFFFFFFFu, (use0 | use1) != 0u)) {
+        uint32_t sv0[32], sv1[32];
+        tmem_ld32(scol + 0, sv0);
+        tmem_ld32(scol + 32, sv1);
+        tmem_ld_wait(sv0);
+        tmem_ld_wait(sv1);
+        // Row max on raw scores (scale > 0), independent chains.
+        float tmax = -INFINITY;
+        if (!s.corr) {
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          // pooled blocks of this chunk that this row must use: video, in range, skipped
-          const int lo = jb + ch * 32;
-          uint32_t video = 0xFFFFFFFFu;
-          if (lo >= M) {
-            video = 0;
-          } else {
-            if (lo + 32 <= P) video = 0;
-            else if (lo < P) video = 0xFFFFFFFFu << (P - lo);
-            if (M - lo < 32) video &= (1u << (M - lo)) - 1u;
+          for (int c = 0; c < 32; c += 4) {
+            m0 = max3f(m0, __uint_as_float(sv0[c]), __uint_as_float(sv0[c + 1]));
+            m1 = max3f(m1, __uint_as_float(sv0[c + 2]), __uint_as_float(sv0[c + 3]));
+            m2 = max3f(m2, __uint_as_float(sv1[c]), __uint_as_float(sv1[c + 1]));
+            m3 = max3f(m3, __uint_as_float(sv1[c + 2]), __uint_as_float(sv1[c + 3]));
           }
-          const uint32_t use = video ? (~rowmask[lo >> 5] & video) : 0u;
+          tmax = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * p.scale_log2;
+        } else {
+          float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float xv = ((use >> c) & 1u) ? fmaf(__uint_as_float(sv[ch][c]), p.scale_log2, kLog2Block)
-                                               : -INFINITY;
-            sv[ch][c] = __float_as_uint(xv);
-            tmax = fmaxf(tmax, xv);
+            m0 = fmaxf(m0, ((use0 >> c) & 1u) ? __uint_as_float(sv0[c]) : -INFINITY);
+            m1 = fmaxf(m1, ((use1 >> c) & 1u) ? __uint_as_float(sv1[c]) : -INFINITY);
+          }
+          const float mraw = fmaxf(m0, m1);
+          if (mraw != -INFINITY) tmax = fmaf(mraw, p.scale_log2, kLog2Block);
+        }
+        // Online softmax with a stale max: O is rescaled only when the running
+        // max grows by more than 2^8; m, l and O always share one reference.
+        const bool need = (m != -INFINITY) && (tmax > m + kRescaleSlack);
+        warp_need = __any_sync(0xFFFFFFFFu, need);
+        alpha = need ? fast_exp2(m - tmax) : 1.0f;
+        if (need || (m == -INFINITY && tmax > m)) m = tmax;
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        const float bias = (s.corr ? kLog2Block : 0.f) - mref;
+        const uint64_t bias2 = f2_pack(bias, bias);
+        uint64_t acc0 = 0ull, acc1 = 0ull, acc2 = 0ull, acc3 = 0ull;
+        if (!s.corr) {
+          // Every column used: no per-element masking.
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint64_t xa = f2_fma(f2_pack(__uint_as_float(sv0[2 * c]), __uint_as_float(sv0[2 * c + 1])),
+                                       scale2, bias2);
+            const uint64_t xb = f2_fma(f2_pack(__uint_as_float(sv1[2 * c]), __uint_as_float(sv1[2 * c + 1])),
+                                       scale2, bias2);
+            float a0, a1, b0, b1;
+            if (c >= 16 - kFmaExpPairs) {
+              exp2_fma_pair(xa, a0, a1);
+              exp2_fma_pair(xb, b0, b1);
+            } else {
+              f2_unpack(xa, a0, a1);
+              f2_unpack(xb, b0, b1);
+              a0 = fast_exp2(a0);
+              a1 = fast_exp2(a1);
+              b0 = fast_exp2(b0);
+              b1 = fast_exp2(b1);
+            }
+            const uint64_t pa = f2_pack(a0, a1), pb = f2_pack(b0, b1);
+            if (c & 1) {
+              acc1 = f2_add(acc1, pa);
+              acc3 = f2_add(acc3, pb);
+            } else {
+              acc0 = f2_add(acc0, pa);
+              acc2 = f2_add(acc2, pb);
+            }
+            pk0[c] = pack_bf16x2(a0, a1);
+            pk1[c] = pack_bf16x2(b0, b1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint64_t xa = f2_fma(f2_pack(__uint_as_float(sv0[2 * c]), __uint_as_float(sv0[2 * c + 1])),
+                                       scale2, bias2);
+            const uint64_t xb = f2_fma(f2_pack(__uint_as_float(sv1[2 * c]), __uint_as_float(sv1[2 * c + 1])),
+                                       scale2, bias2);
+            float a0, a1, b0, b1;
+            f2_unpack(xa, a0, a1);
+            f2_unpack(xb, b0, b1);
+            a0 = ((use0 >> (2 * c)) & 1u) ? fast_exp2(a0) : 0.f;
+            a1 = ((use0 >> (2 * c + 1)) & 1u) ? fast_exp2(a1) : 0.f;
+            b0 = ((use1 >> (2 * c)) & 1u) ? fast_exp2(b0) : 0.f;
+            b1 = ((use1 >> (2 * c + 1)) & 1u) ? fast_exp2(b1) : 0.f;
+            const uint64_t pa = f2_pack(a0, a1), pb = f2_pack(b0, b1);
+            if (c & 1) {
+              acc1 = f2_add(acc1, pa);
+              acc3 = f2_add(acc3, pb);
+            } else {
+              acc0 = f2_add(acc0, pa);
+              acc2 = f2_add(acc2, pb);
+            }
+            pk0[c] = pack_bf16x2(a0, a1);
+            pk1[c] = pack_bf16x2(b0, b1);
           }
         }
+        const uint64_t a = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
+        float s0, s1;
+        f2_unpack(a, s0, s1);
+        l = fmaf(l, alpha, s0 + s1);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          pk0[c] = 0u;
+          pk1[c] = 0u;
+        }
       }
-      // Online softmax with a stale max: rescale O only when the running max
-      // grows by more than 2^8; m, l and O always share the same reference.
-      // tcgen05.ld/st are warp-collective, so the O pass runs when any row of
-      // the warp needs it (alpha = 1 for the others).
-      const bool need = (m != -INFINITY) && (tmax > m + kRescaleSlack);
-      if (__any_sync(0xFFFFFFFFu, need)) {
-        const float alpha = need ? fast_exp2(m - tmax) : 1.0f;
+      tmem_st16(scol + 0, pk0);
+      tmem_st16(scol + 16, pk1);
+      // Every stage n >= 1 waits for PV(n-1) (the n-th commit on OReady).
+      // Waiting each time keeps the parity unambiguous: PV(n-2) is known to
+      // be done, so only phase n-1 can be pending.  The wait sits after this
+      // stage's math, by when PV(n-1) has normally finished.
+      if (n > 0) {
+        ok = mbar_wait(&bars[kBarOReady], (n - 1) & 1, abort_flag, err, 9, p.timeout_ns);
+        if (!ok) break;
+      }
+      // O *= alpha, with no PV in flight: PV(n-1) is done and PV(n) waits
+      // for the arrival below.  tcgen05.ld/st are warp-collective, so the
+      // pass runs when any row of the warp needs it (alpha = 1 for the others).
+      if (warp_need) {
+        tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -570,27 +737,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
           tmem_st32(lane_addr + kColO + c0, o);
         }
-        l *= alpha;
       }
-      if (need || (m == -INFINITY && tmax > m)) m = tmax;
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      // P = 2^(x - m) as bf16 pairs, 16 TMEM columns per 32-key chunk.
-      float rs = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if (ch < nch) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = fast_exp2(__uint_as_float(sv[ch][2 * c]) - mref);
-            const float p1 = fast_exp2(__uint_as_float(sv[ch][2 * c + 1]) - mref);
-            rs += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(lane_addr + kColS + ch * 16, pk);
-        }
-      }
-      l += rs;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[kBarPFull]);

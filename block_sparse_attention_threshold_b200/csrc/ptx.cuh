@@ -64,6 +64,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` pass, instead of spinning and taking issue
+// slots from the warps doing the math.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitHintNs = 20000;  // one sleep of a waiting thread, at most
+
 // Bounded wait for the phase with the given parity to complete.
 //
 // Every wait in the kernels goes through here.  It gives up after
@@ -76,15 +94,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           int* err_word, int site, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
-        *abort = 1;
-        atomicCAS(err_word, 0, site);
-        return false;
-      }
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      atomicCAS(err_word, 0, site);
+      return false;
     }
   }
 }
@@ -264,6 +280,66 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes two fp32 lanes per instruction with the .f32x2 forms; a
+// pair lives in one 64-bit register.
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair on the FMA pipe (no MUFU).  Range reduction in the manner
+// of Cody and Waite: x = n + f with n = round(x) (obtained by adding
+// 1.5 * 2^23, whose low mantissa bits then hold n) and f in [-1/2, 1/2];
+// 2^f ~ 1 + c1 f + c2 f^2 + c3 f^3 with coefficients fitted by least squares
+// of the relative error (fit_exp2_poly.py, max relative error 1.2e-4); 2^n is
+// applied by adding n to the exponent field.  Inputs are clamped at -126 so
+// the exponent never underflows; larger than +64 is never passed here.
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC1 = 0.6933686137199402f, kC2 = 0.24221783876419067f,
+                  kC3 = 0.05459282547235489f;
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));
+  const uint64_t r = f2_add(t, f2_pack(-kMagic, -kMagic));
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
+  q = f2_fma(q, f, f2_pack(kC1, kC1));
+  q = f2_fma(q, f, f2_pack(1.f, 1.f));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(q, q0, q1);
+  // The magic constant's low 9 bits are zero, so (bits(t) << 23) == n << 23.
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
