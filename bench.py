@@ -399,6 +399,80 @@ def run_gpu(args, rank, world, local_rank):
     return result
 
 
+def run_sweep(args):
+    """One JSON line per (workload, tau): kernel times and rates, kept fractions.
+
+    Pool, attend and dense launches are timed alone with CUDA events (median of
+    --reps); the dense-equivalent rate counts one pool + one attend as a step.
+    """
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_threshold_b200 import abi, build, synthetic as syn
+
+    build.build()
+    abi.lib()
+    dev = torch.device("cuda", 0)
+    torch.zeros(1, device=dev)
+    keep_pool_memory(0)
+    names = [args.workload] if args.workload != "all" else [
+        "draft_n16128", "refine_n32768", "long_n65536", "sweep_n131072"]
+    peaks = measured_peaks()
+    for name in names:
+        w = syn.workload(name)
+        qb, kb, vb = syn.generate_bf16(w)
+        q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (qb, kb, vb))
+        del qb, kb, vb
+        out = torch.empty_like(q)
+        nbytes, _ = abi.workspace_layout(w.B, w.H, w.N, w.D)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+        def timed(fn, reps):
+            fn()
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(reps)]
+            for a, b in ev:
+                a.record()
+                fn()
+                b.record()
+            torch.cuda.synchronize()
+            return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+        pool_ms = timed(lambda: abi.pool(q, k, v, ws), args.reps)
+        dense_ms = timed(lambda: abi.dense_forward(q, k, v, out=out), max(1, args.reps // 2))
+        taus = [args.tau] if args.tau is not None else list(w.taus)
+        total = w.B * w.H * w.M * w.M
+        for tau in taus:
+            opts = abi.Opts()
+            cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+            opts.kept_pairs = cnt.data_ptr()
+            opts.exact_pairs = cnt.data_ptr() + 8
+            abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, opts=opts)
+            torch.cuda.synchronize()
+            kept, exact = (int(x) for x in cnt.cpu().tolist())
+            att_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out), args.reps)
+            kept_fl = kept * 4.0 * 64 * 64 * w.D
+            corr_fl = (total - kept) * 4.0 * 64 * w.D
+            step = pool_ms + att_ms
+            row = {
+                "workload": name, "tau": tau, "kept_frac": kept / total, "exact_frac": exact / total,
+                "attend_ms": att_ms, "pool_ms": pool_ms, "dense_ms": dense_ms,
+                "dense_equiv_tflops": w.dense_flops() / step / 1e9,
+                "actual_tflops_kept": kept_fl / att_ms / 1e9,
+                "actual_tflops_kept_plus_corr": (kept_fl + corr_fl) / att_ms / 1e9,
+                "frac_of_peak_kept_plus_corr": (kept_fl + corr_fl) / att_ms / 1e9 / peaks["bf16_tflops"],
+                "tensor_tflops_exact_union": exact * 4.0 * 64 * 64 * w.D / att_ms / 1e9,
+                "dense_tflops": w.dense_flops() / dense_ms / 1e9,
+                "speedup_vs_dense": dense_ms / step,
+                "pool_gbs": (3.0 * w.B * w.H * w.N * w.D * 2 + w.B * w.H * w.M * w.D * 12) / pool_ms / 1e6,
+                "device_status": abi.device_status(),
+            }
+            print(json.dumps(row), flush=True)
+        del q, k, v, out, ws
+        torch.cuda.empty_cache()
+
+
 def run_reference(args, rank):
     from block_sparse_attention_threshold_b200 import synthetic as syn
     if rank != 0:
@@ -449,6 +523,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="kernel table: one JSON line per (workload, tau); --workload all for every one")
+    ap.add_argument("--reps", type=int, default=5, help="timed launches per kernel in --sweep")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -459,6 +536,10 @@ def main():
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torchrun (one rank per GPU)")
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank)
         if res is not None:
