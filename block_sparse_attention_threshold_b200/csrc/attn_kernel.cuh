@@ -93,8 +93,8 @@ struct SmemPlan {
   static constexpr int kMaskB = kMaskA + kMaskWords * 4;
   static constexpr int kMaskU = kMaskB + kMaskWords * 4;
   static constexpr int kQbar = kMaskU + kMaskWords * 4;  // 2 x D floats
-  static constexpr int kRed = kQbar + 2 * D * 4;         // 32 floats
-  static constexpr int kBars = kRed + 32 * 4;
+  static constexpr int kRed = kQbar + 2 * D * 4;         // 64 floats
+  static constexpr int kBars = kRed + 64 * 4;
   static constexpr int kNumBars = 4 * kRingStages + 2 + 6;
   static constexpr int kMisc = kBars + kNumBars * 8;     // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
@@ -151,6 +151,23 @@ struct Stage {
   bool corr;
 };
 
+// Number of stages StageIter yields for these masks, without walking them:
+// popcount of the union plus the correction tiles that are needed.
+__device__ __forceinline__ int count_stages(const uint32_t* mU, const uint32_t* mA, const uint32_t* mB,
+                                            int M, int P, bool dense) {
+  const int nw = (M + 31) >> 5;
+  int n = 0;
+  for (int w = 0; w < nw; ++w) n += __popc(mU[w]);
+  if (dense) return n;
+  for (int c = 0; c < ((M + 63) >> 6); ++c) {
+    uint32_t any = 0u;
+    for (int w = 2 * c; w < 2 * c + 2 && w < nw; ++w)
+      any |= ((~mA[w]) | (~mB[w])) & video_bits(w * 32, M, P);
+    n += any != 0u;
+  }
+  return n;
+}
+
 struct StageIter {
   int j = 0;
   int c = 0;
@@ -185,25 +202,32 @@ struct StageIter {
   }
 };
 
-// Block-wide (128 softmax threads, named barrier 1) sum of two values.
-__device__ __forceinline__ void sm_reduce2(float& a, float& b, float* red, int st) {
+// CTA-wide (all kThreads threads) sum of two values / min-max of two pairs.
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ void cta_reduce2(float& a, float& b, float* red, int tid) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
     b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
   }
-  named_bar_sync(1, 128);
-  if ((st & 31) == 0) {
-    red[(st >> 5) * 2] = a;
-    red[(st >> 5) * 2 + 1] = b;
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    red[(tid >> 5) * 2] = a;
+    red[(tid >> 5) * 2 + 1] = b;
   }
-  named_bar_sync(1, 128);
-  a = red[0] + red[2] + red[4] + red[6];
-  b = red[1] + red[3] + red[5] + red[7];
+  __syncthreads();
+  a = 0.f;
+  b = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    a += red[2 * w];
+    b += red[2 * w + 1];
+  }
 }
 
-__device__ __forceinline__ void sm_reduce_minmax(float& mn_a, float& mx_a, float& mn_b, float& mx_b,
-                                                 float* red, int st) {
+__device__ __forceinline__ void cta_reduce_minmax(float& mn_a, float& mx_a, float& mn_b, float& mx_b,
+                                                  float* red, int tid) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mn_a = fminf(mn_a, __shfl_xor_sync(0xFFFFFFFFu, mn_a, o));
@@ -211,26 +235,31 @@ __device__ __forceinline__ void sm_reduce_minmax(float& mn_a, float& mx_a, float
     mn_b = fminf(mn_b, __shfl_xor_sync(0xFFFFFFFFu, mn_b, o));
     mx_b = fmaxf(mx_b, __shfl_xor_sync(0xFFFFFFFFu, mx_b, o));
   }
-  named_bar_sync(1, 128);
-  if ((st & 31) == 0) {
-    red[16 + (st >> 5) * 4 + 0] = mn_a;
-    red[16 + (st >> 5) * 4 + 1] = mx_a;
-    red[16 + (st >> 5) * 4 + 2] = mn_b;
-    red[16 + (st >> 5) * 4 + 3] = mx_b;
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    float* r = red + 2 * kWarps + (tid >> 5) * 4;
+    r[0] = mn_a;
+    r[1] = mx_a;
+    r[2] = mn_b;
+    r[3] = mx_b;
   }
-  named_bar_sync(1, 128);
-  mn_a = fminf(fminf(red[16], red[20]), fminf(red[24], red[28]));
-  mx_a = fmaxf(fmaxf(red[17], red[21]), fmaxf(red[25], red[29]));
-  mn_b = fminf(fminf(red[18], red[22]), fminf(red[26], red[30]));
-  mx_b = fmaxf(fmaxf(red[19], red[23]), fmaxf(red[27], red[31]));
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float* r = red + 2 * kWarps + w * 4;
+    mn_a = fminf(mn_a, r[0]);
+    mx_a = fmaxf(mx_a, r[1]);
+    mn_b = fminf(mn_b, r[2]);
+    mx_b = fmaxf(mx_b, r[3]);
+  }
 }
 
 // Router: pooled scores of query blocks iA, iB against every video key
-// block, population mean/std, threshold, keep bits.  Runs on the 128
-// softmax threads; scores live in the (not yet used) K/V rings.
+// block, population mean/std, threshold, keep bits.  Runs on all the CTA's
+// threads before the mainloop; scores live in the (not yet used) K/V rings.
 template <int D>
 __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, int iB, bool hasB,
-                                           uint8_t* smem, int st) {
+                                           uint8_t* smem, int tid) {
   using L = SmemPlan<D>;
   uint32_t* mA = reinterpret_cast<uint32_t*>(smem + L::kMaskA);
   uint32_t* mB = reinterpret_cast<uint32_t*>(smem + L::kMaskB);
@@ -244,18 +273,18 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
   if ((videoA || videoB) && nv > 0) {
     const float* qa = p.qbar + (static_cast<size_t>(bh) * M + iA) * D;
     const float* qb = p.qbar + (static_cast<size_t>(bh) * M + (hasB ? iB : iA)) * D;
-    for (int d = st; d < D; d += 128) {
+    for (int d = tid; d < D; d += kThreads) {
       sq[d] = qa[d];
       sq[D + d] = qb[d];
     }
-    named_bar_sync(1, 128);
+    __syncthreads();
     // Scores, 32 key blocks per warp step: lane l holds dims [D/32 * l, +D/32)
     // of every row, so each row is one coalesced load of the warp; the 32
     // partial dot products per lane are then reduced across lanes by a
     // butterfly that leaves row (base + l)'s score in lane l.
     {
       constexpr int kDpl = D / 32;  // dims per lane: 4 (D = 128) or 2 (D = 64)
-      const int lane = st & 31, wq = st >> 5;
+      const int lane = tid & 31, wq = tid >> 5;
       float qa[kDpl], qb[kDpl];
 #pragma unroll
       for (int d = 0; d < kDpl; ++d) {
@@ -263,7 +292,7 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
         qb[d] = sq[D + lane * kDpl + d];
       }
       const float* kb = p.kbar + static_cast<size_t>(bh) * M * D + lane * kDpl;
-      for (int base = P + wq * 32; base < M; base += 128) {
+      for (int base = P + wq * 32; base < M; base += 32 * kWarps) {
         float pa[32], pb[32];
 #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
@@ -310,28 +339,28 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
         }
       }
     }
-    named_bar_sync(1, 128);
+    __syncthreads();
     // Pass 1: mean (and exact-equality check through min/max).
     float sa = 0.f, sb = 0.f;
     float mna = INFINITY, mxa = -INFINITY, mnb = INFINITY, mxb = -INFINITY;
-    for (int j = st; j < nv; j += 128) {
+    for (int j = tid; j < nv; j += kThreads) {
       const float a = sc[j], b = sc[kMaxBlocks + j];
       sa += a; sb += b;
       mna = fminf(mna, a); mxa = fmaxf(mxa, a);
       mnb = fminf(mnb, b); mxb = fmaxf(mxb, b);
     }
-    sm_reduce2(sa, sb, red, st);
-    sm_reduce_minmax(mna, mxa, mnb, mxb, red, st);
+    cta_reduce2(sa, sb, red, tid);
+    cta_reduce_minmax(mna, mxa, mnb, mxb, red, tid);
     const float mua = sa / nv, mub = sb / nv;
     // Pass 2: population variance about the mean.
     float va = 0.f, vb = 0.f;
-    for (int j = st; j < nv; j += 128) {
+    for (int j = tid; j < nv; j += kThreads) {
       const float a = sc[j] - mua, b = sc[kMaxBlocks + j] - mub;
       va = fmaf(a, a, va);
       vb = fmaf(b, b, vb);
     }
-    named_bar_sync(1, 128);  // everyone has read red[] of the previous reduction
-    sm_reduce2(va, vb, red, st);
+    __syncthreads();  // everyone has read red[] of the previous reduction
+    cta_reduce2(va, vb, red, tid);
     const float sda = (mna == mxa) ? 0.f : sqrtf(va / nv);
     const float sdb = (mnb == mxb) ? 0.f : sqrtf(vb / nv);
     const bool allA = (p.tau == -INFINITY) || sda == 0.f;
@@ -339,8 +368,8 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
     const float thrA = mua + p.tau * sda;
     const float thrB = mub + p.tau * sdb;
     // Keep bits, one 32-block word per warp iteration.
-    const int lane = st & 31, wq = st >> 5;
-    for (int w = wq; w < nw; w += 4) {
+    const int lane = tid & 31, wq = tid >> 5;
+    for (int w = wq; w < nw; w += kWarps) {
       const int j = w * 32 + lane;
       bool ka = true, kb2 = true;
       if (j >= M) {
@@ -358,7 +387,7 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
     }
   } else {
     // Prefix query blocks (or no video keys): every block kept.
-    for (int w = st; w < nw; w += 128) {
+    for (int w = tid; w < nw; w += kThreads) {
       const int lo = w * 32;
       const uint32_t full = (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
       mA[w] = full;
@@ -443,35 +472,34 @@ __global__ void __launch_bounds__(kThreads, 2)
                     static_cast<int>(row0 + h * 64));
   }
 
-  if (warp >= 2) {
-    const int st = tid - 64;
-    if (kDense) {
-      for (int w = st; w < nw; w += 128) {
-        const int lo = w * 32;
-        const uint32_t fullw = (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
-        mA[w] = fullw;
-        mB[w] = fullw;
-      }
-    } else {
-      route_tile<D>(p, bh, iA, iB, hasB, smem, st);
+  // Routing on all threads (the producer has already issued the Q load), or
+  // the all-kept mask of the dense kernel.
+  if (kDense) {
+    for (int w = tid; w < nw; w += kThreads) {
+      const int lo = w * 32;
+      const uint32_t fullw = (M - lo >= 32) ? 0xFFFFFFFFu : ((1u << (M - lo)) - 1u);
+      mA[w] = fullw;
+      mB[w] = fullw;
     }
-    named_bar_sync(1, 128);
-    for (int w = st; w < nw; w += 128) mU[w] = mA[w] | mB[w];
-    if (!kDense && (p.debug_mask != nullptr || p.kept_pairs != nullptr || p.exact_pairs != nullptr)) {
-      unsigned long long kept = 0, uni = 0;
-      for (int w = st; w < nw; w += 128) {
-        kept += __popc(mA[w]) + (hasB ? __popc(mB[w]) : 0);
-        uni += __popc(mA[w] | mB[w]) * (hasB ? 2 : 1);
-        if (p.debug_mask != nullptr) {
-          p.debug_mask[(static_cast<size_t>(bh) * M + iA) * nw + w] = mA[w];
-          if (hasB) p.debug_mask[(static_cast<size_t>(bh) * M + iB) * nw + w] = mB[w];
-        }
-      }
-      if (p.kept_pairs != nullptr && kept) atomicAdd(p.kept_pairs, kept);
-      if (p.exact_pairs != nullptr && uni) atomicAdd(p.exact_pairs, uni);
-    }
-    fence_proxy_async_smem();  // scores were written to the rings by generic stores
+  } else {
+    route_tile<D>(p, bh, iA, iB, hasB, smem, tid);
   }
+  __syncthreads();
+  for (int w = tid; w < nw; w += kThreads) mU[w] = mA[w] | mB[w];
+  if (!kDense && (p.debug_mask != nullptr || p.kept_pairs != nullptr || p.exact_pairs != nullptr)) {
+    unsigned long long kept = 0, uni = 0;
+    for (int w = tid; w < nw; w += kThreads) {
+      kept += __popc(mA[w]) + (hasB ? __popc(mB[w]) : 0);
+      uni += __popc(mA[w] | mB[w]) * (hasB ? 2 : 1);
+      if (p.debug_mask != nullptr) {
+        p.debug_mask[(static_cast<size_t>(bh) * M + iA) * nw + w] = mA[w];
+        if (hasB) p.debug_mask[(static_cast<size_t>(bh) * M + iB) * nw + w] = mB[w];
+      }
+    }
+    if (p.kept_pairs != nullptr && kept) atomicAdd(p.kept_pairs, kept);
+    if (p.exact_pairs != nullptr && uni) atomicAdd(p.exact_pairs, uni);
+  }
+  fence_proxy_async_smem();  // scores were written to the rings by generic stores
   __syncthreads();
 
   if (warp == 0) {
@@ -521,12 +549,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kStageKeys, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
-      int total = 0;
-      {
-        StageIter it;
-        Stage s;
-        while (it.next(s, mU, mA, mB, M, P, kDense)) ++total;
-      }
+      const int total = count_stages(mU, mA, mB, M, P, kDense);
       bool ok = mbar_wait(&bars[kBarQ], 0, abort_flag, err, 3, p.timeout_ns);
       // S(n) = Q K(n)^T into S buffer n % 2; A = Q (K-major SW128), B = K.
       auto issue_s = [&](int n) -> bool {
