@@ -33,6 +33,11 @@ Sources (the pages hold prose only; no formula, listing or worked example):
 [S4] "MiniMax 官推背书 Sol Engine" (arex-research 647c3193), section "another
      framing on the same project page: 3.95x near-lossless": rejected blocks get
      a "Taylor approximation" compensation.
+[S5] Sol-H3 DGX Spark release (arex-research 3d0ff631), section "latent
+     hand-off: 384p draft to 768p refine": the draft stage uses sparse attention
+     at 90 % video sparsity in 64-token blocks on cuDNN block-sparse attention,
+     i.e. a fixed budget of video key blocks per query block and no
+     compensation for the dropped ones.
 
 Readings where the pages are silent (each also listed in the design notes):
   * pooling is the arithmetic mean over the block's tokens (count c_j);
@@ -150,9 +155,38 @@ def route(q: np.ndarray, k: np.ndarray, block: int, prefix_len: int, tau: float,
     return Route(score=score, mu=mu, sigma=sigma, thr=thr, keep=keep)
 
 
+def route_budget(q: np.ndarray, k: np.ndarray, block: int, prefix_len: int, keep_blocks: int,
+                 scale: float | None = None) -> Route:
+    """Fixed-budget routing of the draft stage [S5]: every video query block
+    keeps its ``keep_blocks`` highest-scoring video key blocks (same pooled
+    scores as ``route``; ties go to the lower block index), plus the prefix.
+    Prefix query blocks stay dense.  mu/sigma/thr are not used (nan)."""
+    q = _check_head(q)
+    k = _check_head(k)
+    N, D = q.shape
+    if prefix_len % block:
+        raise ValueError("prefix_len must be a whole number of blocks")
+    if keep_blocks < 0:
+        raise ValueError("keep_blocks must be >= 0")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    qbar, _ = pool_blocks(q, block)
+    kbar, _ = pool_blocks(k, block)
+    M = qbar.shape[0]
+    P = prefix_len // block
+    score = scale * (qbar @ kbar.T)
+    keep = np.ones((M, M), dtype=bool)
+    for i in range(P, M):
+        s = score[i, P:]
+        order = np.argsort(-s, kind="stable")  # descending, lower index first on ties
+        keep[i, P:] = False
+        keep[i, P + order[:keep_blocks]] = True
+    nan = np.full(M, np.nan)
+    return Route(score=score, mu=nan, sigma=nan.copy(), thr=nan.copy(), keep=keep)
+
+
 def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, prefix_len: int,
                    tau: float, scale: float | None = None, qblocks=None,
-                   routing: Route | None = None) -> np.ndarray:
+                   routing: Route | None = None, correct: bool = True) -> np.ndarray:
     """Sol-Attn output rows of the listed query blocks of one head.
 
     For each query row r of block i [S1, S3]:
@@ -162,6 +196,8 @@ def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, pref
       out_r = (sum_t e^{l_rt - m} v_t + sum_j e^{l_rj - m} vbar_j)
               / (sum_t e^{l_rt - m} + sum_j e^{l_rj - m}),  m = max of all logits,
     i.e. one softmax over exact and pooled terms together.
+    With ``correct=False`` skipped blocks are dropped instead (plain
+    block-sparse attention, the draft stage of [S5]).
     Returns [len(qblocks) * block, D] (rows of a short last block are omitted).
     """
     q = _check_head(q)
@@ -179,7 +215,7 @@ def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, pref
     for i in qblocks:
         rows = q[i * block:min(N, (i + 1) * block)]
         kept = np.nonzero(r.keep[i])[0]
-        skipped = np.nonzero(~r.keep[i])[0]
+        skipped = np.nonzero(~r.keep[i])[0] if correct else np.zeros(0, dtype=np.int64)
         tok = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in kept]) \
             if len(kept) else np.zeros(0, dtype=np.int64)
         l_exact = scale * (rows @ k[tok].T)

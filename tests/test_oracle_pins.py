@@ -296,3 +296,54 @@ def test_dropping_the_count_weight_would_be_caught():
     den = 64 * np.exp(kv[kept]).sum() + np.exp(kv[skipped]).sum()
     wrong = num / den
     assert abs(wrong - g["expect"]["out_video_row_tau_1.2"]) > 1e-3
+
+
+# ----------------------------------------------------------------------------- fixed budget (draft stage)
+
+def test_budget_route_keeps_the_top_blocks_with_low_index_ties():
+    block = 64
+    # video scores 0.5, 2, 2, 1, 3 (prefix block 0 scores 9): budget 2 keeps
+    # blocks 5 (3.0) and 2 (2.0, lower index than the tied block 3)
+    k = _blocky([9.0, 0.5, 2.0, 2.0, 1.0, 3.0], block)
+    q = np.ones_like(k)
+    r = orc.route_budget(q, k, block, 64, 2, 1.0)
+    for i in range(1, 6):
+        assert list(np.nonzero(r.keep[i])[0]) == [0, 2, 5]
+    assert r.keep[0].all()
+    assert orc.route_budget(q, k, block, 64, 0, 1.0).keep[1:, 1:].sum() == 0
+    assert orc.route_budget(q, k, block, 64, 99, 1.0).keep.all()
+
+
+def test_budget_without_correction_is_attention_over_the_kept_keys():
+    """No correction: each video row attends exactly to the prefix tokens plus
+    its kept blocks' tokens -- textbook attention over that key subset."""
+    w, q, k, v = _tiny_inputs()
+    L, P = w.prefix_len, w.P
+    scale = 1 / math.sqrt(w.D)
+    qh, kh, vh = q[0, 1], k[0, 1], v[0, 1]
+    r = orc.route_budget(qh, kh, 64, L, 3)
+    assert (r.keep[P:, P:].sum(axis=1) == 3).all()
+    for i in (P, P + 5, w.M - 1):
+        tok = np.concatenate([np.arange(j * 64, (j + 1) * 64) for j in np.nonzero(r.keep[i])[0]])
+        ref = _sdpa(qh[i * 64:(i + 1) * 64], kh[tok], vh[tok], scale)
+        out = orc.solattn_blocks(qh, kh, vh, 64, L, 0.0, qblocks=[i], routing=r, correct=False)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    # full budget = dense attention
+    rf = orc.route_budget(qh, kh, 64, L, w.M)
+    out = orc.solattn_blocks(qh, kh, vh, 64, L, 0.0, routing=rf, correct=False)
+    np.testing.assert_allclose(out, _sdpa(qh, kh, vh, scale), rtol=0, atol=1e-12)
+
+
+def test_budget_route_agrees_with_brute_force_ranking():
+    rng = np.random.default_rng(21)
+    N, D, L, kb = 64 * 12, 8, 128, 4
+    q = rng.standard_normal((N, D))
+    k = rng.standard_normal((N, D))
+    r = orc.route_budget(q, k, 64, L, kb)
+    M, P = N // 64, L // 64
+    qb = [[sum(q[t, d] for t in range(i * 64, (i + 1) * 64)) / 64 for d in range(D)] for i in range(M)]
+    kbar = [[sum(k[t, d] for t in range(j * 64, (j + 1) * 64)) / 64 for d in range(D)] for j in range(M)]
+    for i in range(P, M):
+        s = [(sum(a * b for a, b in zip(qb[i], kbar[j])), j) for j in range(P, M)]
+        top = sorted(s, key=lambda x: (-x[0], x[1]))[:kb]
+        assert sorted(j for _, j in top) == [j for j in range(P, M) if r.keep[i, j]]
