@@ -442,21 +442,33 @@ def run_sweep(args):
         pool_ms = timed(lambda: abi.pool(q, k, v, ws), args.reps)
         dense_ms = timed(lambda: abi.dense_forward(q, k, v, out=out), max(1, args.reps // 2))
         taus = [args.tau] if args.tau is not None else list(w.taus)
+        budget = 0
+        if args.budget_sparsity is not None:  # fixed-budget routing, skipped blocks dropped
+            budget = max(1, round((1.0 - args.budget_sparsity) * (w.M - w.P)))
+            taus = [0.0]
         total = w.B * w.H * w.M * w.M
         for tau in taus:
             opts = abi.Opts()
+            opts.budget_blocks = budget
+            opts.skip_correction = 1 if budget else 0
             cnt = torch.zeros(2, dtype=torch.int64, device=dev)
             opts.kept_pairs = cnt.data_ptr()
             opts.exact_pairs = cnt.data_ptr() + 8
             abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, opts=opts)
             torch.cuda.synchronize()
             kept, exact = (int(x) for x in cnt.cpu().tolist())
-            att_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out), args.reps)
+            run_opts = abi.Opts()
+            run_opts.budget_blocks = budget
+            run_opts.skip_correction = 1 if budget else 0
+            att_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, opts=run_opts),
+                           args.reps)
             kept_fl = kept * 4.0 * 64 * 64 * w.D
-            corr_fl = (total - kept) * 4.0 * 64 * w.D
+            corr_fl = 0.0 if budget else (total - kept) * 4.0 * 64 * w.D
             step = pool_ms + att_ms
             row = {
-                "workload": name, "tau": tau, "kept_frac": kept / total, "exact_frac": exact / total,
+                "workload": name, "tau": None if budget else tau,
+                "routing": f"budget {budget} blocks, no correction" if budget else "threshold",
+                "kept_frac": kept / total, "exact_frac": exact / total,
                 "attend_ms": att_ms, "pool_ms": pool_ms, "dense_ms": dense_ms,
                 "dense_equiv_tflops": w.dense_flops() / step / 1e9,
                 "actual_tflops_kept": kept_fl / att_ms / 1e9,
@@ -526,6 +538,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="kernel table: one JSON line per (workload, tau); --workload all for every one")
     ap.add_argument("--reps", type=int, default=5, help="timed launches per kernel in --sweep")
+    ap.add_argument("--budget-sparsity", type=float, default=None,
+                    help="--sweep with fixed-budget routing keeping (1 - s) of the video blocks, "
+                         "skipped blocks dropped (the draft stage's block-sparse attention)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -42,6 +42,8 @@ class Opts(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("timeout_ms", ctypes.c_uint),
         ("test_skip_first_k_load", ctypes.c_int),
+        ("budget_blocks", ctypes.c_int),
+        ("skip_correction", ctypes.c_int),
     ]
 
 

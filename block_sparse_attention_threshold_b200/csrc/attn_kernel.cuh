@@ -79,6 +79,8 @@ struct AttnParams {
   unsigned long long* exact_pairs;  // or null
   uint64_t timeout_ns;
   int skip_first_k_arrival;  // test hook: producer never loads stage 0
+  int budget;                // > 0: keep this many top-scoring video blocks per query block
+  bool correct;              // pooled correction of skipped blocks (else they are dropped)
 };
 
 template <int D>
@@ -94,7 +96,8 @@ struct SmemPlan {
   static constexpr int kMaskU = kMaskB + kMaskWords * 4;
   static constexpr int kQbar = kMaskU + kMaskWords * 4;  // 2 x D floats
   static constexpr int kRed = kQbar + 2 * D * 4;         // 64 floats
-  static constexpr int kBars = kRed + 64 * 4;
+  static constexpr int kHist = kRed + 64 * 4;            // 2 x 256 counters + 8 words (budget routing)
+  static constexpr int kBars = kHist + (2 * 256 + 8) * 4;
   static constexpr int kNumBars = 4 * kRingStages + 2 + 6;
   static constexpr int kMisc = kBars + kNumBars * 8;     // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16;
@@ -143,9 +146,9 @@ __device__ __forceinline__ uint32_t video_bits(int lo, int M, int P) {
 }
 
 // The work of a tile, in order.  Exact stages: every block of the union of
-// the two query blocks' kept sets, ascending.  Correction stages: pooled
-// keys [64c, 64c + 64) holding at least one video block that either query
-// block skipped.
+// the two query blocks' kept sets, ascending.  Correction stages (unless
+// the correction is off): pooled keys [64c, 64c + 64) holding at least one
+// video block that either query block skipped.
 struct Stage {
   int j;      // exact: key block; correction: pooled tile c
   bool corr;
@@ -154,11 +157,11 @@ struct Stage {
 // Number of stages StageIter yields for these masks, without walking them:
 // popcount of the union plus the correction tiles that are needed.
 __device__ __forceinline__ int count_stages(const uint32_t* mU, const uint32_t* mA, const uint32_t* mB,
-                                            int M, int P, bool dense) {
+                                            int M, int P, bool no_corr) {
   const int nw = (M + 31) >> 5;
   int n = 0;
   for (int w = 0; w < nw; ++w) n += __popc(mU[w]);
-  if (dense) return n;
+  if (no_corr) return n;
   for (int c = 0; c < ((M + 63) >> 6); ++c) {
     uint32_t any = 0u;
     for (int w = 2 * c; w < 2 * c + 2 && w < nw; ++w)
@@ -172,7 +175,7 @@ struct StageIter {
   int j = 0;
   int c = 0;
   __device__ __forceinline__ bool next(Stage& s, const uint32_t* mU, const uint32_t* mA,
-                                       const uint32_t* mB, int M, int P, bool dense) {
+                                       const uint32_t* mB, int M, int P, bool no_corr) {
     const int nw = (M + 31) >> 5;
     if (j < M) {
       const int j0 = next_bit(mU, j, nw);
@@ -184,7 +187,7 @@ struct StageIter {
       }
       j = M;
     }
-    if (dense) return false;
+    if (no_corr) return false;
     const int nc = (M + 63) >> 6;
     while (c < nc) {
       const int cc = c++;
@@ -251,6 +254,120 @@ __device__ __forceinline__ void cta_reduce_minmax(float& mn_a, float& mx_a, floa
     mx_a = fmaxf(mx_a, r[1]);
     mn_b = fminf(mn_b, r[2]);
     mx_b = fmaxf(mx_b, r[3]);
+  }
+}
+
+// Order-preserving map of an fp32 score to an unsigned key (larger score,
+// larger key).
+__device__ __forceinline__ uint32_t score_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Fixed-budget routing (draft stage): keep the `budget` highest scores of
+// each video query block, ties at the cut going to the lower block index.
+// The cut is found exactly by a 4-pass, 8-bit radix select over the score
+// keys (shared-memory histograms, one warp picks each digit); a single warp
+// then writes the keep words in block order, which settles ties.
+template <int D>
+__device__ __forceinline__ void route_budget_masks(const AttnParams& p, const float* sc, uint8_t* smem,
+                                                   int tid, bool videoA, bool videoB, bool hasB,
+                                                   uint32_t* mA, uint32_t* mB) {
+  using L = SmemPlan<D>;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L::kHist);  // [2][256]
+  uint32_t* bc = hist + 512;                                      // broadcast words
+  const int M = p.M, P = p.P, nv = M - P;
+  const int nw = (M + 31) >> 5;
+  const int kb = p.budget < nv ? p.budget : nv;
+  uint32_t prefix[2] = {0u, 0u}, pmask = 0u;
+  uint32_t need[2] = {static_cast<uint32_t>(kb), static_cast<uint32_t>(kb)};
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 512; i += kThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int j = tid; j < nv; j += kThreads) {
+      const uint32_t ua = score_key(sc[j]), ub = score_key(sc[kMaxBlocks + j]);
+      if ((ua & pmask) == prefix[0]) atomicAdd(&hist[(ua >> shift) & 255u], 1u);
+      if ((ub & pmask) == prefix[1]) atomicAdd(&hist[256 + ((ub >> shift) & 255u)], 1u);
+    }
+    __syncthreads();
+    const int wq = tid >> 5, lane = tid & 31;
+    if (wq < 2) {
+      // Bins in descending digit order: lane l holds digits 255-8l .. 248-8l.
+      const uint32_t* h = hist + 256 * wq;
+      uint32_t loc[8], lsum = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        loc[i] = h[255 - 8 * lane - i];
+        lsum += loc[i];
+      }
+      uint32_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t run = incl - lsum;  // keys in higher digits than this lane's bins
+      const uint32_t nd = need[wq];
+      int found = -1;
+      uint32_t above = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (found < 0 && run < nd && nd <= run + loc[i]) {
+          found = i;
+          above = run;
+        }
+        run += loc[i];
+      }
+      const uint32_t who = __ballot_sync(0xFFFFFFFFu, found >= 0);
+      if (who != 0u && lane == __ffs(who) - 1) {
+        bc[2 * wq] = static_cast<uint32_t>(255 - 8 * lane - found);
+        bc[2 * wq + 1] = above;
+      }
+    }
+    __syncthreads();
+    for (int q2 = 0; q2 < 2; ++q2) {
+      prefix[q2] |= bc[2 * q2] << shift;
+      need[q2] -= bc[2 * q2 + 1];
+    }
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  // prefix[q] is now the key of the budget-th highest score; need[q] of the
+  // keys equal to it are kept, lowest block first.
+  if ((tid >> 5) == 0) {
+    const int lane = tid & 31;
+    uint32_t left[2] = {need[0], need[1]};
+    for (int w = 0; w < nw; ++w) {
+      const int j = w * 32 + lane;
+      bool ka = j < M, kb2 = j < M;
+      bool ea = false, eb = false;
+      if (j >= P && j < M) {
+        const uint32_t ua = score_key(sc[j - P]), ub = score_key(sc[kMaxBlocks + j - P]);
+        if (videoA) {
+          ka = ua > prefix[0];
+          ea = ua == prefix[0];
+        }
+        if (videoB) {
+          kb2 = ub > prefix[1];
+          eb = ub == prefix[1];
+        }
+      }
+      // ties at the cut: the first `left` of them in block order
+      uint32_t tie = __ballot_sync(0xFFFFFFFFu, ea);
+      const uint32_t rank_a = __popc(tie & ((1u << lane) - 1u));
+      if (ea && rank_a < left[0]) ka = true;
+      left[0] -= min(left[0], static_cast<uint32_t>(__popc(tie)));
+      tie = __ballot_sync(0xFFFFFFFFu, eb);
+      const uint32_t rank_b = __popc(tie & ((1u << lane) - 1u));
+      if (eb && rank_b < left[1]) kb2 = true;
+      left[1] -= min(left[1], static_cast<uint32_t>(__popc(tie)));
+      const uint32_t wa = __ballot_sync(0xFFFFFFFFu, ka);
+      const uint32_t wb = __ballot_sync(0xFFFFFFFFu, kb2);
+      if (lane == 0) {
+        mA[w] = wa;
+        mB[w] = hasB ? wb : wa;
+      }
+    }
   }
 }
 
@@ -340,6 +457,10 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
       }
     }
     __syncthreads();
+    if (p.budget > 0) {
+      route_budget_masks<D>(p, sc, smem, tid, videoA, videoB, hasB, mA, mB);
+      return;
+    }
     // Pass 1: mean (and exact-equality check through min/max).
     float sa = 0.f, sb = 0.f;
     float mna = INFINITY, mxa = -INFINITY, mnb = INFINITY, mxb = -INFINITY;
@@ -429,6 +550,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int iA = 2 * qt, iB = 2 * qt + 1;
   const bool hasB = iB < M;
   const int nw = (M + 31) >> 5;
+  const bool no_corr = kDense || !p.correct;
   int* err = &g_sol_attn_error;
 
   if (tid == 0) {
@@ -511,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       Stage s;
       int n = 0;
       bool ok = true;
-      while (ok && it.next(s, mU, mA, mB, M, P, kDense)) {
+      while (ok && it.next(s, mU, mA, mB, M, P, no_corr)) {
         const int slot = n % kRingStages;
         const uint32_t use_parity = ((n / kRingStages) - 1) & 1;
         const int row = static_cast<int>(s.corr ? prow_head + static_cast<size_t>(s.j) * 64
@@ -549,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kStageKeys, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
-      const int total = count_stages(mU, mA, mB, M, P, kDense);
+      const int total = count_stages(mU, mA, mB, M, P, no_corr);
       bool ok = mbar_wait(&bars[kBarQ], 0, abort_flag, err, 3, p.timeout_ns);
       // S(n) = Q K(n)^T into S buffer n % 2; A = Q (K-major SW128), B = K.
       auto issue_s = [&](int n) -> bool {
@@ -612,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     Stage s;
     int n = 0;
     bool ok = true;
-    while (it.next(s, mU, mA, mB, M, P, kDense)) {
+    while (it.next(s, mU, mA, mB, M, P, no_corr)) {
       const uint32_t scol = lane_addr + 64u * (n & 1);
       ok = mbar_wait(&bars[kBarSFull + (n & 1)], (n >> 1) & 1, abort_flag, err, 7, p.timeout_ns);
       if (!ok) break;

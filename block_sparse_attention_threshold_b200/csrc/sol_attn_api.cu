@@ -115,6 +115,7 @@ int check_io(const void* q, const void* k, const void* v, const void* out) {
 int check_opts(const sol_attn_opts* o) {
   if (o == nullptr) return SOL_ATTN_OK;
   if (!(std::isfinite(o->softmax_scale)) || o->softmax_scale < 0.f) return SOL_ATTN_ERR_INVALID_ARG;
+  if (o->budget_blocks < 0) return SOL_ATTN_ERR_INVALID_ARG;
   return SOL_ATTN_OK;
 }
 
@@ -186,6 +187,8 @@ int launch_attend(const void* q, const void* k, const void* v, void* out, const 
   const unsigned tms = (o != nullptr && o->timeout_ms > 0) ? o->timeout_ms : 1000u;
   p.timeout_ns = static_cast<uint64_t>(tms) * 1000000ull;
   p.skip_first_k_arrival = o ? o->test_skip_first_k_load : 0;
+  p.budget = o ? o->budget_blocks : 0;
+  p.correct = !(o != nullptr && o->skip_correction != 0);
 
   const long long tiles = static_cast<long long>(B) * H * p.tiles_per_head;
   dim3 grid(static_cast<unsigned>(tiles));

@@ -82,6 +82,18 @@ typedef struct {
   /* Test hook, keep 0: the loader skips the first key tile of every CTA so
    * the consumer's bounded wait runs out and the timeout path is exercised. */
   int test_skip_first_k_load;
+  /* 0: routing by threshold (mean + tau * std).  > 0: fixed-budget routing of
+   * the draft stage -- every video query block keeps its `budget_blocks`
+   * highest-scoring video key blocks (same pooled scores; ties at the cut go
+   * to the lower block index; tau is ignored), plus the prefix.  The draft
+   * stage of the pages runs at 90 % video sparsity in 64-token blocks
+   * (Sol-H3 DGX Spark release, section "latent hand-off: 384p draft to 768p
+   * refine").  Must be >= 0. */
+  int budget_blocks;
+  /* Nonzero: skipped blocks are dropped instead of receiving the pooled
+   * correction (plain block-sparse attention, as on the draft stage's
+   * block-sparse backend). */
+  int skip_correction;
 } sol_attn_opts;
 
 /* Sol-Attn forward [R1]-[R4]: pooling, routing, exact attention on kept

@@ -33,12 +33,15 @@ def to_device(*arrays):
             for a in arrays]
 
 
-def run_sol(w, tau, q, k, v, want_mask=True):
+def run_sol(w, tau, q, k, v, want_mask=True, budget=0, correct=True):
     """Sol-Attn on device tensors; returns (out bf16 tensor, keep [B,H,M,M] bool or None,
-    kept_pairs, exact_pairs)."""
+    kept_pairs, exact_pairs).  budget > 0 selects fixed-budget routing;
+    correct=False drops skipped blocks."""
     M = w.M
     dev = q.device
     opts = abi.Opts()
+    opts.budget_blocks = int(budget)
+    opts.skip_correction = 0 if correct else 1
     cnt = torch.zeros(2, dtype=torch.int64, device=dev)
     opts.kept_pairs = cnt.data_ptr()
     opts.exact_pairs = cnt.data_ptr() + 8
@@ -67,10 +70,13 @@ def _blas_single_thread():
         return contextlib.nullcontext()
 
 
-def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False, workers=None):
+def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False, workers=None,
+                   budget=0, correct=True):
     """Compare GPU `out` (and `keep`) with the oracle, head by head in threads.
 
     qblocks: query-block indices to check per head (None = all).
+    budget > 0: fixed-budget routing; mask disagreements are then measured
+    against the cut score (the budget-th highest) instead of the threshold.
     Returns a dict of metrics; raises AssertionError on a violated bound.
     """
     got_all = out.float().cpu().numpy()
@@ -89,17 +95,29 @@ def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False
             ref = orc.dense_rows(q64, k64, v64, rows=rows)
         else:
             r = orc.route(q64, k64, 64, w.prefix_len, tau)
-            ref = orc.solattn_blocks(q64, k64, v64, 64, w.prefix_len, tau, qblocks=blocks, routing=r)
+            cut = r.thr
+            if budget > 0:
+                rb = orc.route_budget(q64, k64, 64, w.prefix_len, budget)
+                P = w.P
+                cut = np.full(w.M, np.nan)
+                for i in range(P, w.M):
+                    sv = np.sort(r.score[i, P:])[::-1]
+                    cut[i] = sv[min(budget, sv.size) - 1]
+                r_use = orc.Route(score=r.score, mu=r.mu, sigma=r.sigma, thr=cut, keep=rb.keep)
+            else:
+                r_use = r
+            ref = orc.solattn_blocks(q64, k64, v64, 64, w.prefix_len, tau, qblocks=blocks, routing=r_use,
+                                     correct=correct)
             if keep is not None:
                 g = keep[b, h]
-                mism = g != r.keep
-                res["pairs"] = r.keep.size
+                mism = g != r_use.keep
+                res["pairs"] = r_use.keep.size
                 res["mismatch"] = int(mism.sum())
                 if res["mismatch"]:
                     ii, jj = np.nonzero(mism)
-                    dist = np.abs(r.score[ii, jj] - r.thr[ii]) / r.sigma[ii]
+                    dist = np.abs(r.score[ii, jj] - cut[ii]) / r.sigma[ii]
                     res["worst_band"] = float(np.nanmax(dist))
-                res["kept"] = int(r.keep.sum())
+                res["kept"] = int(r_use.keep.sum())
         got = got_all[b, h][rows].astype(np.float64)
         res["err2"] = float(np.sum((got - ref) ** 2))
         res["ref2"] = float(np.sum(ref ** 2))

@@ -80,6 +80,9 @@ def test_argument_validation_happens_before_any_device_call(L):
     assert _fwd(L, opts=o) == E.ERR_INVALID_ARG
     o.softmax_scale = math.inf
     assert _fwd(L, opts=o) == E.ERR_INVALID_ARG
+    o.softmax_scale = 0.0
+    o.budget_blocks = -1
+    assert _fwd(L, opts=o) == E.ERR_INVALID_ARG
     # empty problems succeed without doing anything
     assert _fwd(L, B=0) == E.OK
     assert _fwd(L, N=0) == E.OK
