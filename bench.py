@@ -403,7 +403,9 @@ def run_sweep(args):
     """One JSON line per (workload, tau): kernel times and rates, kept fractions.
 
     Pool, attend and dense launches are timed alone with CUDA events (median of
-    --reps); the dense-equivalent rate counts one pool + one attend as a step.
+    --reps launches; attend gets more launches when needed so that its timed
+    region lasts --sweep-min-ms, with SM clocks sampled meanwhile); the
+    dense-equivalent rate counts one pool + one attend as a step.
     """
     import numpy as np
     import torch
@@ -427,9 +429,16 @@ def run_sweep(args):
         nbytes, _ = abi.workspace_layout(w.B, w.H, w.N, w.D)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
 
-        def timed(fn, reps):
+        def timed(fn, reps, min_ms=0.0):
+            # One untimed launch also estimates the duration; short kernels get
+            # more launches so the timed region spans at least min_ms.
+            a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
             fn()
+            b0.record()
             torch.cuda.synchronize()
+            est = max(a0.elapsed_time(b0), 1e-3)
+            reps = max(reps, min(2000, math.ceil(min_ms / est)))
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(reps)]
             for a, b in ev:
@@ -460,8 +469,9 @@ def run_sweep(args):
             run_opts = abi.Opts()
             run_opts.budget_blocks = budget
             run_opts.skip_correction = 1 if budget else 0
-            att_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, opts=run_opts),
-                           args.reps)
+            with ClockSampler(0) as clk:
+                att_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, opts=run_opts),
+                               args.reps, min_ms=args.sweep_min_ms)
             kept_fl = kept * 4.0 * 64 * 64 * w.D
             corr_fl = 0.0 if budget else (total - kept) * 4.0 * 64 * w.D
             step = pool_ms + att_ms
@@ -479,6 +489,7 @@ def run_sweep(args):
                 "speedup_vs_dense": dense_ms / step,
                 "pool_gbs": (3.0 * w.B * w.H * w.N * w.D * 2 + w.B * w.H * w.M * w.D * 12) / pool_ms / 1e6,
                 "device_status": abi.device_status(),
+                "clocks": clk.summary(),
             }
             print(json.dumps(row), flush=True)
         del q, k, v, out, ws
@@ -538,6 +549,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="kernel table: one JSON line per (workload, tau); --workload all for every one")
     ap.add_argument("--reps", type=int, default=5, help="timed launches per kernel in --sweep")
+    ap.add_argument("--sweep-min-ms", type=float, default=500.0,
+                    help="--sweep: lower bound on each attend timing region (more launches if needed)")
     ap.add_argument("--budget-sparsity", type=float, default=None,
                     help="--sweep with fixed-budget routing keeping (1 - s) of the video blocks, "
                          "skipped blocks dropped (the draft stage's block-sparse attention)")
