@@ -668,7 +668,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      // Descriptors are built once.  A ring slot or k-step only moves the
+      // start-address field (shared address >> 4, below 2^14, so adding an
+      // offset never carries): one add per MMA on the issue path, which
+      // shares its SMSP with softmax warps.
+      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(smem_u32(sV), L::kChunkBytes, 1024);
       const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kStageKeys, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
       const int total = count_stages(mU, mA, mB, M, P, no_corr);
@@ -679,14 +685,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&bars[kBarKFull + slot], (n / kRingStages) & 1, abort_flag, err, 4, p.timeout_ns))
           return false;
         tc_fence_after();
-        const uint32_t ka = sKa + slot * L::kBlockBytes;
+        const uint64_t kd = kdesc + static_cast<uint32_t>((slot * L::kBlockBytes) >> 4);
         const uint32_t dcol = tmem + 64u * (n & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = (kk >> 2) * L::kQChunkBytes + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-          mma_bf16_ss(dcol, sdesc_sw128(sQa + qoff, 16, 1024), sdesc_sw128(ka + koff, 16, 1024),
-                      idesc_qk, kk > 0);
+          constexpr int kQStep = L::kQChunkBytes >> 4, kKStep = L::kChunkBytes >> 4;
+          mma_bf16_ss(dcol, qdesc + static_cast<uint32_t>((kk >> 2) * kQStep + (kk & 3) * 2),
+                      kd + static_cast<uint32_t>((kk >> 2) * kKStep + (kk & 3) * 2), idesc_qk, kk > 0);
         }
         mma_commit(&bars[kBarSFull + (n & 1)]);
         mma_commit(&bars[kBarKEmpty + slot]);
@@ -702,10 +707,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         // O += P V: A = P from S buffer n % 2 (TMEM), B = V (MN-major).
         const uint32_t pcol = tmem + 64u * (n & 1);
-        const uint32_t va = sVa + slot * L::kBlockBytes;
+        const uint64_t vd = vdesc + static_cast<uint32_t>((slot * L::kBlockBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kStageKeys / 16; ++kk) {
-          mma_bf16_ts(tmem + kColO, pcol + kk * 8, sdesc_sw128(va + kk * 16 * 128, L::kChunkBytes, 1024),
+          mma_bf16_ts(tmem + kColO, pcol + kk * 8, vd + static_cast<uint32_t>(kk * ((16 * 128) >> 4)),
                       idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars[kBarVEmpty + slot]);
