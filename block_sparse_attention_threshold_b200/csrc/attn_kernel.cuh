@@ -544,9 +544,25 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / p.tiles_per_head;
-  const int qt = blockIdx.x % p.tiles_per_head;
   const int M = p.M, P = p.P;
+  // Launch order: a tile holding a prefix query block attends to every key
+  // block and runs several times longer than a video tile, so the prefix
+  // tiles of all heads come first and the video tiles follow, head by head.
+  // The long tiles then never form the tail of the grid.
+  int bh = static_cast<int>(blockIdx.x) / p.tiles_per_head;
+  int qt = static_cast<int>(blockIdx.x) % p.tiles_per_head;
+  if constexpr (!kDense) {
+    const int T = p.tiles_per_head;
+    const int PT = min(T, (P + 1) / 2);  // tiles holding a prefix query block
+    const int idx = static_cast<int>(blockIdx.x), nlong = p.B * p.H * PT;
+    if (idx < nlong) {
+      bh = idx / PT;
+      qt = idx % PT;
+    } else {
+      bh = (idx - nlong) / (T - PT);
+      qt = PT + (idx - nlong) % (T - PT);
+    }
+  }
   const int iA = 2 * qt, iB = 2 * qt + 1;
   const bool hasB = iB < M;
   const int nw = (M + 31) >> 5;
