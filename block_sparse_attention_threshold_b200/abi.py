@@ -60,6 +60,7 @@ _SIGS = {
     "sol_attn_pool": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "sol_attn_attend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
     "sol_attn_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sol_attn_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sol_attn_device_status": (_I, [_P]),
     "sol_attn_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -151,6 +152,33 @@ def forward_noalloc(q, k, v, tau: float, prefix_len: int = 0, out=None, stream=N
                                         B, H, N, D, block, float(tau), int(prefix_len),
                                         _stream(stream))
     _check(st, "sol_attn_forward_noalloc")
+    return out
+
+
+def forward_host(q, k, v, tau: float, prefix_len: int = 0, out=None, heads_per_chunk: int = 0,
+                 stream=None, block: int = BLOCK):
+    """Sol-Attn through sol_attn_forward_host: q, k, v and out are CPU bf16
+    tensors (page-locked for copy/compute overlap), contiguous [B, H, N, D].
+    The library copies head chunks in, computes and copies them back on its
+    own pipeline; `out` is complete once `stream` (the current CUDA stream by
+    default) has finished."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda:
+            raise TypeError(f"{name} must be a CPU bf16 tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, D]")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    B, H, N, D = (int(x) for x in q.shape)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU bf16 tensor shaped like q")
+    st = lib().sol_attn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     B, H, N, D, block, float(tau), int(prefix_len),
+                                     int(heads_per_chunk), _stream(stream))
+    _check(st, "sol_attn_forward_host")
     return out
 
 

@@ -3,6 +3,7 @@
 // (except sol_attn_device_status).
 #include "sol_attn.h"
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -302,6 +303,100 @@ int sol_attn_dense_forward(const void* q, const void* k, const void* v, void* ou
   if ((st = check_device()) != SOL_ATTN_OK) return st;
   return launch_attend(q, k, v, out, nullptr, B, H, N, D, -INFINITY, 0, nullptr, true,
                        static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int N, int D, int block, float tau, int prefix_len, int heads_per_chunk,
+                          void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if (heads_per_chunk < 0) return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const int BH = B * H;  // B*H*N fits in int (check_shape), so B*H does
+  const int hc = heads_per_chunk > 0 ? std::min(heads_per_chunk, BH) : (BH + 7) / 8;
+  const int nchunks = (BH + hc - 1) / hc;
+  const int nbuf = std::min(3, nchunks);
+  const size_t seq_elems = static_cast<size_t>(N) * D;
+  const size_t tensor_bytes = round256(static_cast<size_t>(hc) * seq_elems * 2);
+  const size_t set_bytes = 4 * tensor_bytes;  // q, k, v, out of one chunk
+  const size_t ws_bytes = sol_attn_workspace_bytes(1, hc, N, D, nullptr);
+
+  uint8_t* dev = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&dev), nbuf * set_bytes + ws_bytes, s) != cudaSuccess)
+    return SOL_ATTN_ERR_CUDA;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr, ev_in[3] = {}, ev_out[3] = {}, ev_free[3] = {};
+  bool ok = cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) == cudaSuccess;
+  for (int b = 0; ok && b < nbuf; ++b)
+    ok = cudaEventCreateWithFlags(&ev_in[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_out[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_free[b], cudaEventDisableTiming) == cudaSuccess;
+  // The copy streams start after the allocation and any earlier work on `stream`.
+  ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess &&
+       cudaStreamWaitEvent(h2d, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(d2h, ev_start, 0) == cudaSuccess;
+  const Workspace w = split_workspace(dev + nbuf * set_bytes, 1, hc, N, D);
+  const uint8_t* hq = static_cast<const uint8_t*>(q);
+  const uint8_t* hk = static_cast<const uint8_t*>(k);
+  const uint8_t* hv = static_cast<const uint8_t*>(v);
+  uint8_t* ho = static_cast<uint8_t*>(out);
+  st = SOL_ATTN_OK;
+  for (int c = 0; ok && st == SOL_ATTN_OK && c < nchunks; ++c) {
+    const int b = c % nbuf;
+    const int heads = std::min(hc, BH - c * hc);
+    const size_t off = static_cast<size_t>(c) * hc * seq_elems * 2, bytes = heads * seq_elems * 2;
+    uint8_t* dq = dev + b * set_bytes;
+    uint8_t* dk = dq + tensor_bytes;
+    uint8_t* dv = dk + tensor_bytes;
+    uint8_t* dout = dv + tensor_bytes;
+    // Buffer set b is free once the copy-back of chunk c - nbuf has finished.
+    if (c >= nbuf) ok = cudaStreamWaitEvent(h2d, ev_free[b], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dq, hq + off, bytes, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaMemcpyAsync(dk, hk + off, bytes, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaMemcpyAsync(dv, hv + off, bytes, cudaMemcpyHostToDevice, h2d) == cudaSuccess &&
+         cudaEventRecord(ev_in[b], h2d) == cudaSuccess && cudaStreamWaitEvent(s, ev_in[b], 0) == cudaSuccess;
+    if (!ok) break;
+    st = launch_pool(dq, dk, dv, w, 1, heads, N, D, s);
+    if (st == SOL_ATTN_OK)
+      st = launch_attend(dq, dk, dv, dout, &w, 1, heads, N, D, tau, prefix_len, nullptr, false, s);
+    ok = st == SOL_ATTN_OK && cudaEventRecord(ev_out[b], s) == cudaSuccess &&
+         cudaStreamWaitEvent(d2h, ev_out[b], 0) == cudaSuccess &&
+         cudaMemcpyAsync(ho + off, dout, bytes, cudaMemcpyDeviceToHost, d2h) == cudaSuccess &&
+         cudaEventRecord(ev_free[b], d2h) == cudaSuccess;
+  }
+  // Whatever happened above, `stream` resumes only after both copy streams
+  // have drained (h2d's tail is folded into d2h), and only then is the
+  // scratch released.  If that ordering cannot be enqueued, wait here.
+  const bool tail = ev_start && ev_done && h2d && d2h && cudaEventRecord(ev_start, h2d) == cudaSuccess &&
+                    cudaStreamWaitEvent(d2h, ev_start, 0) == cudaSuccess &&
+                    cudaEventRecord(ev_done, d2h) == cudaSuccess &&
+                    cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
+  if (!tail) {
+    if (h2d) cudaStreamSynchronize(h2d);
+    if (d2h) cudaStreamSynchronize(d2h);
+    ok = false;
+  }
+  if (cudaFreeAsync(dev, s) != cudaSuccess) ok = false;
+  // Streams and events are released by the runtime once their work completes.
+  for (int b = 0; b < 3; ++b) {
+    if (ev_in[b]) cudaEventDestroy(ev_in[b]);
+    if (ev_out[b]) cudaEventDestroy(ev_out[b]);
+    if (ev_free[b]) cudaEventDestroy(ev_free[b]);
+  }
+  if (ev_start) cudaEventDestroy(ev_start);
+  if (ev_done) cudaEventDestroy(ev_done);
+  if (h2d) cudaStreamDestroy(h2d);
+  if (d2h) cudaStreamDestroy(d2h);
+  if (st != SOL_ATTN_OK) return st;
+  return ok ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
 }
 
 int sol_attn_device_status(void* stream) {

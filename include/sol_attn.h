@@ -172,6 +172,31 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
                              int H, int N, int D, int block, float tau, int prefix_len,
                              void* stream);
 
+/* Host-buffer variant of sol_attn_forward: q, k, v and out are HOST
+ * pointers, same [B][H][N][D] bf16 layout and the same result.  The pages
+ * have no counterpart; this is the end-to-end path for a caller whose data
+ * lives in host memory.
+ * Every (b, h) sequence is an independent problem, so the B*H sequences are
+ * cut into chunks of `heads_per_chunk` consecutive ones (0 picks
+ * ceil(B*H / 8); the last chunk may be shorter).  Chunk c's host-to-device
+ * copy runs on an internal copy stream while chunk c-1 is pooled and
+ * attended on `stream` and chunk c-2 is copied back on a second internal
+ * stream; three device buffer sets rotate.
+ *  - Host memory should be page-locked (cudaHostAlloc or cudaHostRegister)
+ *    for the copies to overlap the kernels; pageable memory gives the same
+ *    result without the overlap.
+ *  - Device scratch: three chunk buffer sets of q, k, v, out plus one pooling
+ *    workspace, allocated with cudaMallocAsync on `stream` and freed there.
+ *  - The call returns once all work is enqueued; `out` is complete once
+ *    `stream` has finished it.  The caller must keep the host buffers alive
+ *    and unmodified until then.
+ *  - Argument errors return before anything is enqueued; a CUDA error in
+ *    the middle returns SOL_ATTN_ERR_CUDA and may leave earlier chunks
+ *    enqueued.  heads_per_chunk < 0 is SOL_ATTN_ERR_INVALID_ARG. */
+int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int N, int D, int block, float tau, int prefix_len, int heads_per_chunk,
+                          void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * kernels set when a bounded wait gives up.  SOL_ATTN_OK if none did,
  * SOL_ATTN_ERR_DEVICE_TIMEOUT if one did, SOL_ATTN_ERR_CUDA if the

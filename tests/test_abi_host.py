@@ -22,7 +22,7 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = abi.declared_symbols(HEADER)
-    assert len(names) == 9
+    assert len(names) == 10
     out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -91,6 +91,15 @@ def test_argument_validation_happens_before_any_device_call(L):
     assert L.sol_attn_pool(FAKE, FAKE, FAKE, FAKE + 16, 1, 1, 64, 64, None) == E.ERR_INVALID_ARG
     assert L.sol_attn_attend(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 64, 64, 64, 1.0, 0, None,
                              None) == E.ERR_INVALID_ARG
+    # host-buffer entry point: same checks, plus the chunk size
+    def host(hq=FAKE, heads=0, D=64, tau=1.0, B=1):
+        return L.sol_attn_forward_host(hq, FAKE, FAKE, FAKE, B, 2, 128, D, 64, tau, 0, heads, None)
+    assert host(heads=-1) == E.ERR_INVALID_ARG
+    assert host(hq=0) == E.ERR_INVALID_ARG
+    assert host(hq=FAKE + 8) == E.ERR_INVALID_ARG
+    assert host(D=96) == E.ERR_UNSUPPORTED
+    assert host(tau=math.nan) == E.ERR_INVALID_ARG
+    assert host(B=0) == E.OK
 
 
 def test_python_binding_rejects_non_cuda_tensors(L):
@@ -98,6 +107,8 @@ def test_python_binding_rejects_non_cuda_tensors(L):
     x = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         abi.forward(x, x, x, 1.0)
+    with pytest.raises(TypeError):  # the host entry point wants bf16 CPU tensors
+        abi.forward_host(x.float(), x, x, 1.0)
 
 
 def test_unpack_mask_bit_order():
