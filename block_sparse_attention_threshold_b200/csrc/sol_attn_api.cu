@@ -318,7 +318,13 @@ int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const int BH = B * H;  // B*H*N fits in int (check_shape), so B*H does
-  const int hc = heads_per_chunk > 0 ? std::min(heads_per_chunk, BH) : (BH + 7) / 8;
+  // Default chunk: about 8 MiB of each tensor (one head at N = 32768,
+  // D = 128), enough for full-speed copies while keeping the pipeline's
+  // fill and drain short.
+  const size_t seq_bytes = static_cast<size_t>(N) * D * 2;
+  const int hc = heads_per_chunk > 0
+                     ? std::min(heads_per_chunk, BH)
+                     : static_cast<int>(std::min<size_t>(BH, std::max<size_t>(1, ((8u << 20) + seq_bytes - 1) / seq_bytes)));
   const int nchunks = (BH + hc - 1) / hc;
   const int nbuf = std::min(3, nchunks);
   const size_t seq_elems = static_cast<size_t>(N) * D;

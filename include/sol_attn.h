@@ -177,8 +177,9 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
  * have no counterpart; this is the end-to-end path for a caller whose data
  * lives in host memory.
  * Every (b, h) sequence is an independent problem, so the B*H sequences are
- * cut into chunks of `heads_per_chunk` consecutive ones (0 picks
- * ceil(B*H / 8); the last chunk may be shorter).  Chunk c's host-to-device
+ * cut into chunks of `heads_per_chunk` consecutive ones (0 picks about
+ * 8 MiB of each tensor per chunk, at least one sequence and at most B*H; the
+ * last chunk may be shorter).  Chunk c's host-to-device
  * copy runs on an internal copy stream while chunk c-1 is pooled and
  * attended on `stream` and chunk c-2 is copied back on a second internal
  * stream; three device buffer sets rotate.
