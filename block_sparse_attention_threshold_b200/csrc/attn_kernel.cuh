@@ -376,7 +376,7 @@ __device__ __forceinline__ void route_budget_masks(const AttnParams& p, const fl
 // threads before the mainloop; scores live in the (not yet used) K/V rings.
 template <int D>
 __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, int iB, bool hasB,
-                                           uint8_t* smem, int tid) {
+                                           uint8_t* smem, int tid, float pre_a, float pre_b) {
   using L = SmemPlan<D>;
   uint32_t* mA = reinterpret_cast<uint32_t*>(smem + L::kMaskA);
   uint32_t* mB = reinterpret_cast<uint32_t*>(smem + L::kMaskB);
@@ -388,11 +388,11 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
   const bool videoA = iA >= P, videoB = hasB && iB >= P;
 
   if ((videoA || videoB) && nv > 0) {
-    const float* qa = p.qbar + (static_cast<size_t>(bh) * M + iA) * D;
-    const float* qb = p.qbar + (static_cast<size_t>(bh) * M + (hasB ? iB : iA)) * D;
-    for (int d = tid; d < D; d += kThreads) {
-      sq[d] = qa[d];
-      sq[D + d] = qb[d];
+    // The pooled queries were loaded at kernel entry (thread d holds dim d).
+    static_assert(D <= kThreads, "one pooled-query dimension per thread");
+    if (tid < D) {
+      sq[tid] = pre_a;
+      sq[D + tid] = pre_b;
     }
     __syncthreads();
     // Scores, 32 key blocks per warp step: lane l holds dims [D/32 * l, +D/32)
@@ -569,6 +569,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool no_corr = kDense || !p.correct;
   int* err = &g_sol_attn_error;
 
+  // The router's pooled queries are loaded first thing, so their global
+  // latency overlaps the barrier, TMEM and Q-tile setup below.
+  float pre_qa = 0.f, pre_qb = 0.f;
+  if (!kDense && tid < D && p.qbar != nullptr && ((iA >= P) || (hasB && iB >= P)) && M > P) {
+    pre_qa = __ldg(p.qbar + (static_cast<size_t>(bh) * M + iA) * D + tid);
+    pre_qb = __ldg(p.qbar + (static_cast<size_t>(bh) * M + (hasB ? iB : iA)) * D + tid);
+  }
   if (tid == 0) {
     for (int i = 0; i < kRingStages; ++i) {
       mbar_init(&bars[kBarKFull + i], 1);
@@ -620,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mB[w] = fullw;
     }
   } else {
-    route_tile<D>(p, bh, iA, iB, hasB, smem, tid);
+    route_tile<D>(p, bh, iA, iB, hasB, smem, tid, pre_qa, pre_qb);
   }
   __syncthreads();
   for (int w = tid; w < nw; w += kThreads) mU[w] = mA[w] | mB[w];
