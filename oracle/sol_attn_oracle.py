@@ -39,6 +39,13 @@ Sources (the pages hold prose only; no formula, listing or worked example):
      i.e. a fixed budget of video key blocks per query block and no
      compensation for the dropped ones.
 
+[S6] [S3]'s page, same section, the "fused operators" item: the residual +
+     RMSNorm + modulation, QKNorm + partial RoPE and SwiGLU chains keep their
+     intermediates in registers or on chip; and the kocpc.com.tw report of the
+     same release (www.kocpc.com.tw/?p=668110), section "技術組成：Sol Engine ×
+     Sol-Attn 完整堆疊": the lossless kernel work fuses QKNorm + RoPE among
+     others to cut HBM round trips.  The pages name the chain only.
+
 Readings where the pages are silent (each also listed in the design notes):
   * pooling is the arithmetic mean over the block's tokens (count c_j);
   * the block score uses pooled queries: s_ij = scale * <qbar_i, kbar_j>,
@@ -273,3 +280,60 @@ def dense(q, k, v, scale: float | None = None, rows=None) -> np.ndarray:
     B, H, N, D = q.shape
     out = [dense_rows(q[b, h], k[b, h], v[b, h], scale, rows) for b in range(B) for h in range(H)]
     return np.stack(out).reshape(B, H, -1, D)
+
+
+# ---------------------------------------------------------------------------
+# QKNorm + partial RoPE in front of the pooling [S6].  The pages name the
+# chain and nothing else; the readings:
+#   * QKNorm is RMSNorm over the head dimension of each q (and k) row, with a
+#     per-dimension weight: y = x / sqrt(mean(x^2) + eps) * w;
+#   * "partial" RoPE rotates the first R (rope_dims) dimensions of the row and
+#     leaves the rest, pairing dimension i with i + R/2 ("rotate half") for
+#     i < R/2, by the angle pos * base^(-2 i / R);
+#   * pos is the token's index in its (b, h) sequence, prefix included;
+#   * the kernel writes the result as bf16, and the pooled summaries are the
+#     block means of those bf16 values (what a separate pooling pass over the
+#     written tensors would compute).
+
+
+def rms_norm(x: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm of each row over the last dimension [S6 "QKNorm"]: x / sqrt(mean(x^2) + eps) * w."""
+    x = _check_head(x)
+    w = np.asarray(w, dtype=np.float64)
+    if w.shape != (x.shape[1],):
+        raise ValueError("weight must have one entry per dimension")
+    rms = np.sqrt(np.mean(x * x, axis=1, keepdims=True) + float(eps))
+    return x / rms * w
+
+
+def partial_rope(x: np.ndarray, rope_dims: int, base: float = 10000.0, positions=None) -> np.ndarray:
+    """Rotary embedding of the first ``rope_dims`` dimensions of each row [S6 "partial RoPE"].
+
+    Rows are positions 0..N-1 unless ``positions`` is given.  For i < R/2 the
+    pair (x_i, x_{i+R/2}) is rotated by theta = pos * base^(-2 i / R):
+    (a, b) -> (a cos theta - b sin theta, a sin theta + b cos theta).
+    Dimensions R..D-1 are returned unchanged.
+    """
+    x = _check_head(x)
+    N, D = x.shape
+    R = int(rope_dims)
+    if R < 0 or R > D or R % 2:
+        raise ValueError("rope_dims must be even and within [0, D]")
+    y = x.copy()
+    if R == 0:
+        return y
+    pos = np.arange(N, dtype=np.float64) if positions is None else np.asarray(positions, dtype=np.float64)
+    half = R // 2
+    for i in range(half):
+        theta = pos * float(base) ** (-2.0 * i / R)
+        c, s_ = np.cos(theta), np.sin(theta)
+        a, b = x[:, i], x[:, i + half]
+        y[:, i] = a * c - b * s_
+        y[:, i + half] = a * s_ + b * c
+    return y
+
+
+def qknorm_rope(x: np.ndarray, w: np.ndarray, eps: float, rope_dims: int, base: float = 10000.0):
+    """The fused chain for one head: RMSNorm, then partial RoPE [S6]."""
+    return partial_rope(rms_norm(x, w, eps), rope_dims, base)
+

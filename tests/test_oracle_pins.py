@@ -347,3 +347,51 @@ def test_budget_route_agrees_with_brute_force_ranking():
         s = [(sum(a * b for a, b in zip(qb[i], kbar[j])), j) for j in range(P, M)]
         top = sorted(s, key=lambda x: (-x[0], x[1]))[:kb]
         assert sorted(j for _, j in top) == [j for j in range(P, M) if r.keep[i, j]]
+
+
+# --------------------------------------------------------------------------- QKNorm + partial RoPE
+
+def test_rms_norm_hand_values():
+    # Row [3, 4]: mean square 12.5, so with eps = 0 the row becomes [3, 4] / 3.5355339...
+    # = [0.8485281374238570, 1.1313708498984760] (computed by hand), times the weights.
+    y = orc.rms_norm(np.array([[3.0, 4.0]]), np.array([1.0, 2.0]), 0.0)
+    assert y[0, 0] == pytest.approx(0.8485281374238570, abs=1e-15)
+    assert y[0, 1] == pytest.approx(2.0 * 1.1313708498984760, abs=1e-15)
+
+
+def test_rms_norm_constant_row_closed_form():
+    # A constant row c normalises to c / sqrt(c^2 + eps) in every dimension.
+    c, eps = -3.0, 1e-6
+    w = np.arange(1.0, 9.0)
+    y = orc.rms_norm(np.full((1, 8), c), w, eps)
+    assert np.allclose(y[0], w * (c / math.sqrt(c * c + eps)), rtol=0, atol=1e-15)
+
+
+def test_rope_hand_values():
+    # D = R = 4, base 10000: pair (0, 2) turns by pos * 1, pair (1, 3) by pos * 0.01.
+    x = np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0], [0, 0, 0, 1.0]])
+    y = orc.partial_rope(x, 4, 10000.0, positions=[1, 2, 3])
+    # pos 1, e0: (cos 1, sin 1) on dims (0, 2)
+    assert np.allclose(y[0], [0.5403023058681398, 0, 0.8414709848078965, 0], atol=1e-15)
+    # pos 2, e1: angle 0.02 on dims (1, 3)
+    assert np.allclose(y[1], [0, 0.9998000066665778, 0, 0.01999866669333308], atol=1e-15)
+    # pos 3, e3 (second member of pair (1, 3)): (-sin 0.03, cos 0.03) on dims (1, 3)
+    assert np.allclose(y[2], [0, -0.02999550020249566, 0, 0.9995500337489875], atol=1e-15)
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(7)
+    N, D, R = 40, 16, 8
+    x = rng.normal(size=(N, D))
+    y = orc.partial_rope(x, R, 10000.0)
+    assert np.array_equal(y[0], x[0])                    # position 0 is the identity
+    assert np.array_equal(y[:, R:], x[:, R:])            # dimensions past R untouched
+    for i in range(R // 2):                              # each rotated pair keeps its length
+        assert np.allclose(np.hypot(y[:, i], y[:, i + R // 2]), np.hypot(x[:, i], x[:, i + R // 2]),
+                           rtol=1e-13)
+    # Relative position: <rope(a, m), rope(b, n)> depends on m - n only.
+    a, b = rng.normal(size=D), rng.normal(size=D)
+    m, n = 29, 11
+    lhs = orc.partial_rope(a[None], D, positions=[m])[0] @ orc.partial_rope(b[None], D, positions=[n])[0]
+    rhs = orc.partial_rope(a[None], D, positions=[m - n])[0] @ b
+    assert lhs == pytest.approx(rhs, rel=1e-12)
