@@ -494,6 +494,61 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_prep(args):
+    """QKNorm + partial RoPE ahead of Sol-Attn: the fused pass that also fills
+    the pooled workspace, against the same chain without pooling followed by
+    the standalone pooling pass.  One JSON line; CUDA-event medians."""
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_threshold_b200 import abi, build, synthetic as syn
+
+    build.build()
+    abi.lib()
+    dev = torch.device("cuda", 0)
+    w = syn.workload(args.workload)
+    qb, kb, vb = syn.generate_bf16(w)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (qb, kb, vb))
+    del qb, kb, vb
+    rng = np.random.default_rng(w.seed + 7)
+    wq = torch.from_numpy((1.0 + 0.25 * rng.normal(size=w.D)).astype(np.float32)).to(dev)
+    wk = torch.from_numpy((1.0 + 0.25 * rng.normal(size=w.D)).astype(np.float32)).to(dev)
+    R = args.rope_dims if args.rope_dims is not None else w.D // 2
+    q_out, k_out = torch.empty_like(q), torch.empty_like(k)
+    nbytes, _ = abi.workspace_layout(w.B, w.H, w.N, w.D)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    fused_ms = timed(lambda: abi.qknorm_rope_pool(q, k, v, wq, wk, R, q_out=q_out, k_out=k_out, workspace=ws),
+                     max(10, args.reps))
+    chain_ms = timed(lambda: abi.qknorm_rope_pool(q, k, v, wq, wk, R, q_out=q_out, k_out=k_out, pool=False),
+                     max(10, args.reps))
+    pool_ms = timed(lambda: abi.pool(q_out, k_out, v, ws), max(10, args.reps))
+    elems = w.B * w.H * w.N * w.D
+    fused_bytes = 3 * elems * 2 + 2 * elems * 2 + w.B * w.H * w.M * w.D * 12
+    peaks = measured_peaks()
+    gbs = fused_bytes / (fused_ms * 1e-3) / 1e9
+    row = {
+        "workload": w.name, "rope_dims": R,
+        "fused_ms": fused_ms, "chain_only_ms": chain_ms, "pool_ms": pool_ms,
+        "separate_ms": chain_ms + pool_ms, "saved_ms": chain_ms + pool_ms - fused_ms,
+        "fused_bytes": fused_bytes, "fused_gbs": gbs, "fused_hbm_frac": gbs / peaks["hbm_gbs"],
+        "hbm_peak_gbs": peaks["hbm_gbs"], "device_status": abi.device_status(),
+    }
+    print(json.dumps(row), flush=True)
+
+
 def run_reference(args, rank):
     from block_sparse_attention_threshold_b200 import synthetic as syn
     if rank != 0:
@@ -547,6 +602,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="kernel table: one JSON line per (workload, tau); --workload all for every one")
     ap.add_argument("--reps", type=int, default=5, help="timed launches per kernel in --sweep")
+    ap.add_argument("--prep", action="store_true",
+                    help="time the fused QKNorm + partial RoPE + pooling pass against the unfused pair")
+    ap.add_argument("--rope-dims", type=int, default=None, help="--prep: rotated dimensions (default D/2)")
     ap.add_argument("--sweep-min-ms", type=float, default=500.0,
                     help="--sweep: lower bound on each attend timing region (more launches if needed)")
     ap.add_argument("--budget-sparsity", type=float, default=None,
@@ -565,6 +623,10 @@ def main():
     if args.sweep:
         if rank == 0:
             run_sweep(args)
+        return
+    if args.prep:
+        if rank == 0:
+            run_prep(args)
         return
     if args.impl == "reference":
         res = run_reference(args, rank)

@@ -61,6 +61,7 @@ _SIGS = {
     "sol_attn_attend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
     "sol_attn_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "sol_attn_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "sol_attn_qknorm_rope_pool": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
     "sol_attn_device_status": (_I, [_P]),
     "sol_attn_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -180,6 +181,35 @@ def forward_host(q, k, v, tau: float, prefix_len: int = 0, out=None, heads_per_c
                                      int(heads_per_chunk), _stream(stream))
     _check(st, "sol_attn_forward_host")
     return out
+
+
+def qknorm_rope_pool(q_in, k_in, v, q_weight, k_weight, rope_dims: int, eps: float = 1e-6,
+                     rope_base: float = 10000.0, q_out=None, k_out=None, workspace=None, pool: bool = True,
+                     stream=None):
+    """QKNorm + partial RoPE of q and k through sol_attn_qknorm_rope_pool, with the
+    pooled workspace for sol_attn_attend filled in the same pass (pool=True).
+    q_weight, k_weight: CUDA fp32 [D].  Returns (q_out, k_out, workspace or None)."""
+    import torch
+    B, H, N, D = _shape(q_in, k_in, v)
+    for name, t in (("q_weight", q_weight), ("k_weight", k_weight)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda or t.shape != (D,):
+            raise TypeError(f"{name} must be a CUDA fp32 tensor of shape [D]")
+    q_out = _out_like(q_in, q_out)
+    k_out = _out_like(k_in, k_out)
+    ws_ptr = None
+    if pool:
+        if workspace is None:
+            nbytes, _ = workspace_layout(B, H, N, D)
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q_in.device)
+        ws_ptr = workspace.data_ptr()
+    else:
+        workspace = None
+    st = lib().sol_attn_qknorm_rope_pool(q_in.data_ptr(), k_in.data_ptr(), v.data_ptr(), q_weight.data_ptr(),
+                                         k_weight.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), ws_ptr,
+                                         B, H, N, D, int(rope_dims), float(eps), float(rope_base),
+                                         _stream(stream))
+    _check(st, "sol_attn_qknorm_rope_pool")
+    return q_out, k_out, workspace
 
 
 def noalloc_max_workspace() -> int:

@@ -16,6 +16,7 @@
 
 #include "attn_kernel.cuh"
 #include "pool_kernel.cuh"
+#include "prep_kernel.cuh"
 
 namespace {
 
@@ -403,6 +404,55 @@ int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out
   if (d2h) cudaStreamDestroy(d2h);
   if (st != SOL_ATTN_OK) return st;
   return ok ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+}
+
+int sol_attn_qknorm_rope_pool(const void* q_in, const void* k_in, const void* v, const float* q_weight,
+                              const float* k_weight, void* q_out, void* k_out, void* workspace, int B, int H,
+                              int N, int D, int rope_dims, float eps, float rope_base, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return SOL_ATTN_OK;
+  if (st != SOL_ATTN_OK) return st;
+  if (!q_in || !k_in || !q_out || !k_out || !q_weight || !k_weight || !aligned16(q_in) || !aligned16(k_in) ||
+      !aligned16(q_out) || !aligned16(k_out) || !aligned16(q_weight) || !aligned16(k_weight))
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if (workspace != nullptr &&
+      (!v || !aligned16(v) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return SOL_ATTN_ERR_INVALID_ARG;
+  const bool pow2 = rope_dims > 0 && ((rope_dims / 16) & (rope_dims / 16 - 1)) == 0;
+  if (rope_dims < 0 || rope_dims > D || rope_dims % 16 != 0 || (rope_dims > 0 && !pow2))
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps <= 0.f || !std::isfinite(rope_base) || rope_base <= 1.f)
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  sol::PrepParams pp{};
+  pp.q_in = static_cast<const __nv_bfloat16*>(q_in);
+  pp.k_in = static_cast<const __nv_bfloat16*>(k_in);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.wq = q_weight;
+  pp.wk = k_weight;
+  pp.q_out = static_cast<__nv_bfloat16*>(q_out);
+  pp.k_out = static_cast<__nv_bfloat16*>(k_out);
+  if (workspace != nullptr) {
+    const Workspace w = split_workspace(workspace, B, H, N, D);
+    pp.pool = sol::PoolOut{w.qbar, w.kbar, w.kbar_bf16, w.vbar_bf16};
+  }
+  pp.M = N / SOL_ATTN_BLOCK;
+  pp.rope_dims = rope_dims;
+  pp.eps = eps;
+  for (int i = 0; i < rope_dims / 2; ++i)
+    pp.inv_freq[i] = std::pow(static_cast<double>(rope_base), -2.0 * i / rope_dims);
+  const unsigned nblk = static_cast<unsigned>(static_cast<long long>(B) * H * pp.M);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (workspace != nullptr) {
+    dim3 grid(nblk, 3);
+    if (D == 128) sol::prep_kernel<128, true><<<grid, 128, 0, s>>>(pp);
+    else sol::prep_kernel<64, true><<<grid, 128, 0, s>>>(pp);
+  } else {
+    dim3 grid(nblk, 2);
+    if (D == 128) sol::prep_kernel<128, false><<<grid, 128, 0, s>>>(pp);
+    else sol::prep_kernel<64, false><<<grid, 128, 0, s>>>(pp);
+  }
+  return cudaGetLastError() == cudaSuccess ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
 }
 
 int sol_attn_device_status(void* stream) {

@@ -22,6 +22,8 @@
  *       "3.95x near-lossless": skipped blocks get a Taylor-approximation
  *       compensation; this library implements its zeroth-order term
  *       (count-weighted mean-key logit + ln c_j, mean value).
+ *  [R5] [R3]'s page, same section, fused-operators item: the QKNorm +
+ *       partial RoPE chain keeps its intermediates in registers or on chip.
  *
  * Conventions shared by every entry point
  *  - q, k, v, out: DEVICE pointers to contiguous bf16 arrays laid out
@@ -197,6 +199,27 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
 int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int N, int D, int block, float tau, int prefix_len, int heads_per_chunk,
                           void* stream);
+
+/* QKNorm + partial RoPE of q and k, with the block pooling fused in [R5].
+ * The pages name the chain only; this entry point fixes it as follows.
+ * For every row x of q_in (and of k_in, with k_weight):
+ *   y = x * rsqrt(mean(x^2) + eps) * q_weight          (RMSNorm over D)
+ *   then for i < R/2, R = rope_dims, pos = token index in its sequence:
+ *   (y_i, y_{i+R/2}) <- (y_i c - y_{i+R/2} s, y_i s + y_{i+R/2} c),
+ *   c, s = cos, sin of pos * rope_base^(-2 i / R); dimensions >= R unchanged.
+ * The results are written as bf16 to q_out and k_out.  If `workspace` is not
+ * NULL, the same pass also fills it as sol_attn_pool(q_out, k_out, v) would,
+ * bit for bit, so sol_attn_attend can follow without a separate pooling pass
+ * over HBM; v is then required.  With workspace NULL only q_out and k_out are
+ * written.
+ *   q_weight, k_weight: DEVICE fp32 [D], 16-byte aligned.
+ *   rope_dims: 0, or 16 * 2^k <= D (16, 32, 64 or 128).
+ *   eps > 0 and finite; rope_base > 1 and finite.
+ *   q_out and k_out must not overlap any input or each other.
+ * Same shape rules as the other entry points; asynchronous on `stream`. */
+int sol_attn_qknorm_rope_pool(const void* q_in, const void* k_in, const void* v, const float* q_weight,
+                              const float* k_weight, void* q_out, void* k_out, void* workspace, int B, int H,
+                              int N, int D, int rope_dims, float eps, float rope_base, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word that
  * kernels set when a bounded wait gives up.  SOL_ATTN_OK if none did,

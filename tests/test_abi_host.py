@@ -22,7 +22,7 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = abi.declared_symbols(HEADER)
-    assert len(names) == 10
+    assert len(names) == 11
     out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -100,6 +100,22 @@ def test_argument_validation_happens_before_any_device_call(L):
     assert host(D=96) == E.ERR_UNSUPPORTED
     assert host(tau=math.nan) == E.ERR_INVALID_ARG
     assert host(B=0) == E.OK
+    # QKNorm + RoPE + pooling: rope_dims, eps, base and pointer checks
+    def prep(R=64, eps=1e-6, base=1e4, ws=None, v=FAKE, w=FAKE, D=128, N=128):
+        return L.sol_attn_qknorm_rope_pool(FAKE, FAKE, v, w, FAKE, FAKE, FAKE, ws, 1, 2, N, D, R, eps, base, None)
+    assert prep(R=48) == E.ERR_INVALID_ARG         # 48 / 16 = 3 is not a power of two
+    assert prep(R=8) == E.ERR_INVALID_ARG          # not a multiple of 16
+    assert prep(R=256) == E.ERR_INVALID_ARG        # more than D
+    assert prep(R=-16) == E.ERR_INVALID_ARG
+    assert prep(eps=0.0) == E.ERR_INVALID_ARG
+    assert prep(eps=math.nan) == E.ERR_INVALID_ARG
+    assert prep(base=1.0) == E.ERR_INVALID_ARG
+    assert prep(base=math.inf) == E.ERR_INVALID_ARG
+    assert prep(w=0) == E.ERR_INVALID_ARG          # null weight
+    assert prep(ws=FAKE + 16) == E.ERR_INVALID_ARG  # workspace not 256-byte aligned
+    assert prep(ws=FAKE, v=0) == E.ERR_INVALID_ARG  # pooling needs v
+    assert prep(D=96) == E.ERR_UNSUPPORTED
+    assert prep(N=0) == E.OK
 
 
 def test_python_binding_rejects_non_cuda_tensors(L):
