@@ -22,7 +22,7 @@
  *       "3.95x near-lossless": skipped blocks get a Taylor-approximation
  *       compensation; this library implements its zeroth-order term
  *       (count-weighted mean-key logit + ln c_j, mean value).
- *  [R5] [R3]'s page, same section, fused-operators item: the QKNorm +
+ *  [R6] [R3]'s page, same section, fused-operators item: the QKNorm +
  *       partial RoPE chain keeps its intermediates in registers or on chip.
  *
  * Conventions shared by every entry point
@@ -200,7 +200,7 @@ int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out
                           int N, int D, int block, float tau, int prefix_len, int heads_per_chunk,
                           void* stream);
 
-/* QKNorm + partial RoPE of q and k, with the block pooling fused in [R5].
+/* QKNorm + partial RoPE of q and k, with the block pooling fused in [R6].
  * The pages name the chain only; this entry point fixes it as follows.
  * For every row x of q_in (and of k_in, with k_weight):
  *   y = x * rsqrt(mean(x^2) + eps) * q_weight          (RMSNorm over D)
