@@ -36,11 +36,19 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
 
 
 def kernel_source_hash() -> str:
+    """Hash of the attention kernel's code with comments and blank lines
+    stripped: it ties a stored ncu traffic figure to the code it was taken
+    on, and a comment edit does not invalidate it."""
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "block_sparse_attention_threshold_b200", "csrc")
     for f in ("attn_kernel.cuh", "ptx.cuh"):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        text = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 

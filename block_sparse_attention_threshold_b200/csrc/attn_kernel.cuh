@@ -31,11 +31,15 @@
 //             next block's scores are computed while the softmax works on the
 //             current one; then O += P V with P read from TMEM (P overwrites
 //             its S buffer in place as bf16);
-//  warps 2-5  router (scores, mean/std, keep bits in shared memory), then
-//             online softmax (one TMEM lane = one query row), conditional O
+//  warps 2-5  online softmax (one TMEM lane = one query row), conditional O
 //             rescale, and the epilogue O / l -> bf16.
+//  all warps  route first (pooled scores, mean/std, keep bits in shared
+//             memory); the two pooled queries are loaded at kernel entry.
 // TMEM per CTA: S0 (64 columns) | S1 (64) | O (D) in 256 columns, so two
 // CTAs share an SM.
+// Grid: one CTA per tile; the tiles holding prefix query blocks (dense rows,
+// several times longer) of all heads come first, then the video tiles head
+// by head.
 // The tile visits the union of its two query blocks' kept sets; a row whose
 // block did not keep a visited key block masks it out and gets that block's
 // pooled correction instead.
