@@ -1,6 +1,8 @@
 // Host side of the C ABI declared in include/sol_attn.h: argument checks,
-// workspace, TMA descriptors and kernel launches.  No torch, no host syncs
-// (except sol_attn_device_status).
+// workspace, TMA descriptors, kernel launches and the host-buffer pipeline.
+// No torch.  No host syncs, except in sol_attn_device_status and on the error
+// path of sol_attn_forward_host (when the stream ordering of its tail cannot
+// be enqueued, it drains its own streams before freeing the scratch).
 #include "sol_attn.h"
 
 #include <algorithm>
