@@ -36,7 +36,8 @@
  *  - B, H or N equal to 0 is an empty problem: SOL_ATTN_OK, nothing runs.
  *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous with respect to the host and issues no host
- *    synchronisation, except sol_attn_device_status().
+ *    synchronisation, except sol_attn_device_status() and the error path of
+ *    sol_attn_forward_host() (see there).
  *  - Arguments are validated before any work is enqueued; a call that
  *    returns an error has enqueued nothing.  The library holds no state
  *    besides per-device cached attributes and one device error word.
@@ -195,7 +196,9 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
  *    and unmodified until then.
  *  - Argument errors return before anything is enqueued; a CUDA error in
  *    the middle returns SOL_ATTN_ERR_CUDA and may leave earlier chunks
- *    enqueued.  heads_per_chunk < 0 is SOL_ATTN_ERR_INVALID_ARG. */
+ *    enqueued (if their ordering before the scratch release cannot be
+ *    enqueued either, the call synchronises its internal streams first).
+ *    heads_per_chunk < 0 is SOL_ATTN_ERR_INVALID_ARG. */
 int sol_attn_forward_host(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int N, int D, int block, float tau, int prefix_len, int heads_per_chunk,
                           void* stream);
