@@ -48,6 +48,17 @@ def test_host_entry_matches_device_entry_bit_for_bit(heads_per_chunk, pinned):
     assert torch.equal(out.view(torch.int16), ref.cpu().view(torch.int16))
 
 
+def test_host_entry_d64_matches_device_entry():
+    w, (qb, kb, vb) = _random_inputs(1, 3, 1024, 64, seed=20261105)
+    q, k, v = parity.to_device(qb, kb, vb)
+    ref = abi.forward(q, k, v, 0.5, w.prefix_len)
+    hq, hk, hv = _host(qb, kb, vb)
+    out = abi.forward_host(hq, hk, hv, 0.5, w.prefix_len, heads_per_chunk=2)
+    torch.cuda.synchronize()
+    assert abi.device_status() == abi.OK
+    assert torch.equal(out.view(torch.int16), ref.cpu().view(torch.int16))
+
+
 def test_host_entry_parity_tiny():
     w = syn.workload("tiny_n1024")
     qb, kb, vb = syn.generate_bf16(w)

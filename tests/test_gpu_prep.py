@@ -75,6 +75,22 @@ def test_chain_matches_oracle_and_pool_is_bit_identical(D, R):
     assert none is None and torch.equal(q2, q_out) and torch.equal(k2, k_out)
 
 
+def test_batched_odd_heads():
+    B, H, N, D, R = 2, 3, 512, 128, 32
+    (qb, kb, vb), wq, wk = _inputs(B, H, N, D, seed=20261231)
+    q, k, v = parity.to_device(qb, kb, vb)
+    dev = q.device
+    q_out, k_out, ws = abi.qknorm_rope_pool(q, k, v, torch.from_numpy(wq).to(dev), torch.from_numpy(wk).to(dev),
+                                            R, 1e-5, 500000.0)
+    torch.cuda.synchronize()
+    _check_chain(qb, wq, q_out, R, 1e-5, 500000.0)
+    _check_chain(kb, wk, k_out, R, 1e-5, 500000.0)
+    ref_ws = torch.empty_like(ws)
+    abi.pool(q_out, k_out, v, ref_ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ws, ref_ws)
+
+
 def test_attention_on_fused_workspace_equals_forward():
     w = syn.workload("draft_n16128")
     B, H, N, D = 1, 4, 4096, 128
