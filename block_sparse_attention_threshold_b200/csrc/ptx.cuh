@@ -342,8 +342,4 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& p0, float& p1)
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 }  // namespace sol
