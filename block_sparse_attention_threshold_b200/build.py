@@ -11,7 +11,11 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsolattn.so")
 SOURCES = ["sol_attn_api.cu"]
-DEPS = ["sol_attn_api.cu", "attn_kernel.cuh", "pool_kernel.cuh", "ptx.cuh"]
+
+
+def deps() -> list:
+    """Every CUDA source and header under csrc/, so an edit to any of them rebuilds."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 
 
 def nvcc() -> str:
@@ -32,8 +36,8 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "sol_attn.h")]
-    return all(os.path.getmtime(d) <= t for d in deps)
+    files = [os.path.join(CSRC, d) for d in deps()] + [os.path.join(ROOT, "include", "sol_attn.h")]
+    return all(os.path.getmtime(d) <= t for d in files)
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:

@@ -1,8 +1,10 @@
 // Host side of the C ABI declared in include/sol_attn.h: argument checks,
 // workspace, TMA descriptors, kernel launches and the host-buffer pipeline.
-// No torch.  No host syncs, except in sol_attn_device_status and on the error
-// path of sol_attn_forward_host (when the stream ordering of its tail cannot
-// be enqueued, it drains its own streams before freeing the scratch).
+// No torch.  No host syncs, except in sol_attn_device_status and in
+// sol_attn_forward_host: on its error path (when the stream ordering of its
+// tail cannot be enqueued, it drains its own streams before freeing the
+// scratch), and when `out` is pageable host memory (the runtime then makes
+// each device-to-host copy return only once it has finished).
 #include "sol_attn.h"
 
 #include <algorithm>

@@ -36,8 +36,9 @@
  *  - B, H or N equal to 0 is an empty problem: SOL_ATTN_OK, nothing runs.
  *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Every call is asynchronous with respect to the host and issues no host
- *    synchronisation, except sol_attn_device_status() and the error path of
- *    sol_attn_forward_host() (see there).
+ *    synchronisation, except sol_attn_device_status(), and
+ *    sol_attn_forward_host() on its error path or with a pageable `out`
+ *    (see there).
  *  - Arguments are validated before any work is enqueued; a call that
  *    returns an error has enqueued nothing.  The library holds no state
  *    besides per-device cached attributes and one device error word.
@@ -149,8 +150,10 @@ int sol_attn_attend(const void* q, const void* k, const void* v, void* out,
                     const void* workspace, int B, int H, int N, int D, int block, float tau,
                     int prefix_len, const sol_attn_opts* opts, void* stream);
 
-/* Largest workspace sol_attn_forward_noalloc can serve: 64 MiB, i.e.
- * B*H*N <= 2,796,202 tokens at D = 128 (5,592,405 at D = 64). */
+/* Largest workspace sol_attn_forward_noalloc can serve: 64 MiB.  In whole
+ * 64-token blocks that is B*H*(N/64) <= 43,690 at D = 128 (2,796,160 tokens)
+ * and <= 87,381 at D = 64 (5,592,384 tokens; the workspace then fills the
+ * array exactly). */
 #define SOL_ATTN_NOALLOC_MAX_WORKSPACE (64u << 20)
 
 /* Allocation-free variant of sol_attn_forward, for callers that cannot
@@ -188,7 +191,10 @@ int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* 
  * stream; three device buffer sets rotate.
  *  - Host memory should be page-locked (cudaHostAlloc or cudaHostRegister)
  *    for the copies to overlap the kernels; pageable memory gives the same
- *    result without the overlap.
+ *    result without the overlap.  With a pageable `out` the CUDA runtime
+ *    makes each device-to-host copy return only once it has finished, so
+ *    the call then blocks the host until the last chunk is back (an
+ *    exception to the "no host synchronisation" rule above).
  *  - Device scratch: three chunk buffer sets of q, k, v, out plus one pooling
  *    workspace, allocated with cudaMallocAsync on `stream` and freed there.
  *  - The call returns once all work is enqueued; `out` is complete once

@@ -4,7 +4,9 @@ and compare it with the CPU fp64 oracle on the same seeded inputs.
 Tolerances (the operator's acceptance bar):
   * keep mask: >= 99.9 % of (query block, key block) pairs agree, and every
     disagreement lies within 1e-3 * sigma_i of its threshold (fp32 routing on
-    the GPU vs fp64 in the oracle);
+    the GPU vs fp64 in the oracle); a disagreement where the oracle's answer
+    is forced (prefix rows or columns, tau = -inf, rows whose scores are all
+    equal) fails outright;
   * output: relative L2 error <= 1e-2 and max abs error <= 2e-2 versus fp64
     on the bf16 inputs.
 """
@@ -113,10 +115,21 @@ def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False
                 mism = g != r_use.keep
                 res["pairs"] = r_use.keep.size
                 res["mismatch"] = int(mism.sum())
+                res["hard_mismatch"] = 0
                 if res["mismatch"]:
                     ii, jj = np.nonzero(mism)
-                    dist = np.abs(r.score[ii, jj] - cut[ii]) / r.sigma[ii]
-                    res["worst_band"] = float(np.nanmax(dist))
+                    # A disagreement is only admissible at a routed pair
+                    # (video query block, video key block) whose row has a
+                    # finite cut and a positive spread.  Everywhere else the
+                    # oracle's answer is forced (prefix rows and columns,
+                    # tau = -inf, all scores equal), so any mismatch fails.
+                    P = w.P
+                    sig = r.sigma[ii]
+                    ok = (ii >= P) & (jj >= P) & np.isfinite(cut[ii]) & np.isfinite(sig) & (sig > 0)
+                    res["hard_mismatch"] = int((~ok).sum())
+                    if ok.any():
+                        dist = np.abs(r.score[ii[ok], jj[ok]] - cut[ii[ok]]) / sig[ok]
+                        res["worst_band"] = float(dist.max())
                 res["kept"] = int(r_use.keep.sum())
         got = got_all[b, h][rows].astype(np.float64)
         res["err2"] = float(np.sum((got - ref) ** 2))
@@ -137,6 +150,7 @@ def oracle_compare(w, tau, qb, kb, vb, out, keep=None, qblocks=None, dense=False
         m["mask_agree"] = 1.0 - mism / pairs
         m["mask_mismatch"] = mism
         m["worst_band"] = max((r.get("worst_band", 0.0) for r in results), default=0.0)
+        m["hard_mismatch"] = sum(r["hard_mismatch"] for r in results)
         m["oracle_kept"] = sum(r["kept"] for r in results)
     return m
 
@@ -147,3 +161,4 @@ def assert_parity(m):
     if "mask_agree" in m:
         assert m["mask_agree"] >= MASK_AGREE, m
         assert m["worst_band"] <= MASK_BAND, m
+        assert m["hard_mismatch"] == 0, m

@@ -167,10 +167,9 @@ def test_workload_parity(name):
 def test_sparsity_sweep_parity():
     w = syn.workload("sweep_n131072")
     bits, (q, k, v) = inputs(w)
+    blocks = syn.sample_query_blocks(w.M, w.P, 64, w.seed + 1)
     for tau in w.taus:
-        dense = tau == -math.inf
         out, keep, kept, _ = parity.run_sol(w, tau, q, k, v)
-        blocks = syn.sample_query_blocks(w.M, w.P, 8 if dense else 32, w.seed + 1)
         m = parity.oracle_compare(w, tau, *bits, out, keep, qblocks=blocks)
         print("sweep tau", tau, m, "kept frac", kept / keep.size)
         parity.assert_parity(m)

@@ -395,3 +395,32 @@ def test_rope_invariants():
     lhs = orc.partial_rope(a[None], D, positions=[m])[0] @ orc.partial_rope(b[None], D, positions=[n])[0]
     rhs = orc.partial_rope(a[None], D, positions=[m - n])[0] @ b
     assert lhs == pytest.approx(rhs, rel=1e-12)
+
+
+def test_qknorm_rope_composition_order_hand_values():
+    # The chain is RMSNorm (with its weight) first, then RoPE.  With D = R = 2,
+    # w = [1, 2], eps = 0, the row [1, 0] at position 1 normalises to
+    # [1, 0] / sqrt(1/2) * [1, 2] = [sqrt 2, 0] and then turns by 1 radian:
+    # [sqrt 2 cos 1, sqrt 2 sin 1].  Applying the weight after the rotation
+    # would give [sqrt 2 cos 1, 2 sqrt 2 sin 1]; rotating first and then
+    # normalising with the weight gives the same wrong value, so this pins the
+    # order.  Row 0 (position 0) is not rotated: [1, 0] -> [sqrt 2, 0] as well.
+    x = np.array([[1.0, 0.0], [1.0, 0.0]])
+    y = orc.qknorm_rope(x, np.array([1.0, 2.0]), 0.0, 2)
+    r2 = math.sqrt(2.0)
+    assert np.allclose(y[0], [r2, 0.0], rtol=0, atol=1e-15)
+    assert np.allclose(y[1], [r2 * 0.5403023058681398, r2 * 0.8414709848078965], rtol=0, atol=1e-15)
+    wrong = [r2 * 0.5403023058681398, 2 * r2 * 0.8414709848078965]
+    assert not np.allclose(y[1], wrong, atol=1e-3)
+
+
+def test_qknorm_rope_weight_inside_rotation_pair():
+    # A non-uniform weight on a rotated pair separates "weight, then rotate"
+    # from "rotate, then weight": for x = [0, 1] at position 1 with w = [3, 1],
+    # the normalised row is [0, sqrt 2] (the weight meets a zero), so the
+    # rotation gives [-sqrt 2 sin 1, sqrt 2 cos 1]; weighting after the
+    # rotation would scale the first entry by 3.
+    x = np.array([[0.0, 1.0], [0.0, 1.0]])
+    y = orc.qknorm_rope(x, np.array([3.0, 1.0]), 0.0, 2)
+    r2 = math.sqrt(2.0)
+    assert np.allclose(y[1], [-r2 * 0.8414709848078965, r2 * 0.5403023058681398], rtol=0, atol=1e-15)
