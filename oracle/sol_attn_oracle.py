@@ -191,9 +191,60 @@ def route_budget(q: np.ndarray, k: np.ndarray, block: int, prefix_len: int, keep
     return Route(score=score, mu=nan, sigma=nan.copy(), thr=nan.copy(), keep=keep)
 
 
+def block_cross_moment(k: np.ndarray, v: np.ndarray, block: int = BLOCK):
+    """Centred key/value cross moments of every block, for the first-order
+    term of the Taylor compensation [S4]:
+        Cov_j = (1 / c_j) * sum_t (k_t - kbar_j) (v_t - vbar_j)^T   (D x D).
+    Returns [M, D, D]."""
+    k = _check_head(k)
+    v = _check_head(v)
+    N, D = k.shape
+    kbar, counts = pool_blocks(k, block)
+    vbar, _ = pool_blocks(v, block)
+    out = np.empty((kbar.shape[0], D, v.shape[1]))
+    for j in range(kbar.shape[0]):
+        sl = slice(j * block, min(N, (j + 1) * block))
+        out[j] = (k[sl] - kbar[j]).T @ (v[sl] - vbar[j]) / counts[j]
+    return out
+
+
+def taylor_block_terms(q_rows: np.ndarray, k_blk: np.ndarray, v_blk: np.ndarray, scale: float,
+                       order: int = 0, q_expand=None):
+    """Compensation of one skipped block for the given query rows [S4]: the
+    Taylor expansion of its exact terms around the pooled key kbar.
+
+    Exact:   den = sum_t e^{s q.k_t},   num = sum_t e^{s q.k_t} v_t.
+    With k_t = kbar + d_t (sum_t d_t = 0) and e^{s q.d_t} ~ 1 + s q.d_t:
+      order 0:  den = c e^{s q.kbar},  num = c e^{s q.kbar} vbar;
+      order 1:  den unchanged (its first-order term is s q.sum_t d_t = 0),
+                num = c e^{s q.kbar} (vbar + s Cov^T q),
+                Cov = (1/c) sum_t d_t (v_t - vbar)^T.
+    ``q_expand`` (rows x D, default the rows themselves) is the query used in
+    the first-order term: passing the block's pooled query gives the cheaper
+    per-block-pair form.  Returns (den [rows], num [rows, D]) without any
+    max subtraction (small examples only).
+    """
+    q_rows = np.atleast_2d(np.asarray(q_rows, dtype=np.float64))
+    k_blk = _check_head(k_blk)
+    v_blk = _check_head(v_blk)
+    c = k_blk.shape[0]
+    kbar = k_blk.mean(axis=0)
+    vbar = v_blk.mean(axis=0)
+    w = c * np.exp(scale * (q_rows @ kbar))
+    num = w[:, None] * vbar[None, :]
+    if order >= 1:
+        cov = (k_blk - kbar).T @ (v_blk - vbar) / c
+        qe = q_rows if q_expand is None else np.atleast_2d(np.asarray(q_expand, dtype=np.float64))
+        num = num + w[:, None] * (scale * (qe @ cov))
+    if order > 1:
+        raise ValueError("orders 0 and 1 only")
+    return w, num
+
+
 def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, prefix_len: int,
                    tau: float, scale: float | None = None, qblocks=None,
-                   routing: Route | None = None, correct: bool = True) -> np.ndarray:
+                   routing: Route | None = None, correct: bool = True, order: int = 0,
+                   pooled_query_term: bool = False) -> np.ndarray:
     """Sol-Attn output rows of the listed query blocks of one head.
 
     For each query row r of block i [S1, S3]:
@@ -205,6 +256,10 @@ def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, pref
     i.e. one softmax over exact and pooled terms together.
     With ``correct=False`` skipped blocks are dropped instead (plain
     block-sparse attention, the draft stage of [S5]).
+    ``order=1`` adds the first-order term of the compensation (see
+    ``taylor_block_terms``): skipped block j's value becomes
+    vbar_j + scale * Cov_j^T q_r, or with ``pooled_query_term`` the block's
+    pooled query qbar_i in place of q_r; its weight is unchanged.
     Returns [len(qblocks) * block, D] (rows of a short last block are omitted).
     """
     q = _check_head(q)
@@ -216,6 +271,10 @@ def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, pref
     kbar, counts = pool_blocks(k, block)
     vbar, _ = pool_blocks(v, block)
     M = kbar.shape[0]
+    if order not in (0, 1):
+        raise ValueError("orders 0 and 1 only")
+    cov = block_cross_moment(k, v, block) if (order == 1 and correct) else None
+    qbar = pool_blocks(q, block)[0] if pooled_query_term else None
     if qblocks is None:
         qblocks = range(M)
     outs = []
@@ -231,6 +290,10 @@ def solattn_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, pref
         w_exact = np.exp(l_exact - m[:, None])
         w_pool = np.exp(l_pool - m[:, None])
         num = w_exact @ v[tok] + w_pool @ vbar[skipped]
+        if cov is not None:
+            qe = np.broadcast_to(qbar[i], rows.shape) if pooled_query_term else rows
+            for col, j in enumerate(skipped):
+                num += w_pool[:, col:col + 1] * (scale * (qe @ cov[j]))
         den = w_exact.sum(axis=1) + w_pool.sum(axis=1)
         outs.append(num / den[:, None])
     return np.concatenate(outs, axis=0) if outs else np.zeros((0, D))

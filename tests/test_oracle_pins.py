@@ -424,3 +424,121 @@ def test_qknorm_rope_weight_inside_rotation_pair():
     y = orc.qknorm_rope(x, np.array([3.0, 1.0]), 0.0, 2)
     r2 = math.sqrt(2.0)
     assert np.allclose(y[1], [-r2 * 0.8414709848078965, r2 * 0.5403023058681398], rtol=0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- first-order Taylor compensation
+
+def test_taylor_first_order_hand_values():
+    # Two keys k = kbar +- a u with kbar = 0, u = e0, a = 0.1; values e0 and e1;
+    # q = e0, scale 1.  By hand: Cov = (1/2) sum_t d_t (v_t - vbar)^T
+    # = (a/2) u (v1 - v2)^T = [[0.05, -0.05], [0, 0]], so Cov^T q = [0.05, -0.05];
+    # weight c e^{q.kbar} = 2; order 0 gives num = 2 vbar = [1, 1], order 1
+    # gives 2 ([0.5, 0.5] + [0.05, -0.05]) = [1.1, 0.9].  The exact sum is
+    # e^{0.1} e0 + e^{-0.1} e1 = [1.1051709180756477, 0.9048374180359595].
+    k = np.array([[0.1, 0.0], [-0.1, 0.0]])
+    v = np.array([[1.0, 0.0], [0.0, 1.0]])
+    q = np.array([[1.0, 0.0]])
+    w0, n0 = orc.taylor_block_terms(q, k, v, 1.0, order=0)
+    w1, n1 = orc.taylor_block_terms(q, k, v, 1.0, order=1)
+    assert w0[0] == pytest.approx(2.0) and w1[0] == pytest.approx(2.0)
+    assert np.allclose(n0[0], [1.0, 1.0], atol=1e-15)
+    assert np.allclose(n1[0], [1.1, 0.9], atol=1e-15)
+    # a transposed moment (Cov q instead of Cov^T q) would give [1.1, 1.0]
+    assert not np.allclose(n1[0], [1.1, 1.0], atol=1e-3)
+    exact = np.exp(k @ q[0]) @ v
+    assert np.allclose(exact, [1.1051709180756477, 0.9048374180359595], atol=1e-15)
+    assert np.abs(n1[0] - exact).max() < np.abs(n0[0] - exact).max() / 10
+
+
+def test_taylor_error_orders_by_convergence():
+    # Keys kbar + alpha * d_t: the numerator error of order 0 falls like
+    # alpha, that of order 1 like alpha^2; the denominator error of both like
+    # alpha^2 (its first-order term is zero).
+    rng = np.random.default_rng(11)
+    c, D = 64, 16
+    kbar = rng.normal(size=D) * 0.3
+    d = rng.normal(size=(c, D))
+    d -= d.mean(axis=0)
+    v = rng.normal(size=(c, D)) + 0.5 * d[:, :1]  # values correlated with the key offsets
+    q = rng.normal(size=(3, D))
+    s = 1.0 / math.sqrt(D)
+
+    def errs(alpha, order):
+        k = kbar + alpha * d
+        den, num = orc.taylor_block_terms(q, k, v, s, order=order)
+        e = np.exp(s * (q @ k.T))
+        return np.abs(num - e @ v).max(), np.abs(den - e.sum(axis=1)).max()
+
+    a = 0.02
+    n0a, d0a = errs(a, 0)
+    n0b, d0b = errs(a / 2, 0)
+    n1a, d1a = errs(a, 1)
+    n1b, d1b = errs(a / 2, 1)
+    assert 1.8 < n0a / n0b < 2.2          # first order error of the zeroth-order term
+    assert 3.6 < n1a / n1b < 4.4          # second order once the first-order term is in
+    assert 3.6 < d0a / d0b < 4.4 and d1a == d0a
+
+
+def test_taylor_first_order_reduces_to_zeroth_for_identical_keys():
+    rng = np.random.default_rng(12)
+    B, H, N, D, L = 1, 1, 64 * 10, 16, 128
+    q = rng.normal(size=(N, D))
+    k = np.repeat(rng.normal(size=(N // 64, D)), 64, axis=0)
+    v = rng.normal(size=(N, D))
+    k[:L] = rng.normal(size=(L, D))
+    r = orc.route(q, k, 64, L, 1.0)
+    assert not r.keep.all()
+    o0 = orc.solattn_blocks(q, k, v, 64, L, 1.0, routing=r)
+    o1 = orc.solattn_blocks(q, k, v, 64, L, 1.0, routing=r, order=1)
+    assert np.allclose(o0, o1, rtol=0, atol=1e-14)
+    # ... where identical values too make both exact
+    v2 = np.repeat(rng.normal(size=(N // 64, D)), 64, axis=0)
+    v2[:L] = rng.normal(size=(L, D))
+    o1 = orc.solattn_blocks(q, k, v2, 64, L, 1.0, routing=r, order=1)
+    assert np.allclose(o1, orc.dense_rows(q, k, v2), rtol=0, atol=1e-12)
+
+
+def test_taylor_pooled_query_form_matches_per_row_form_on_constant_rows():
+    # With every query row of a block equal, the pooled query is that row and
+    # the cheaper per-block-pair form is the per-row form.
+    rng = np.random.default_rng(13)
+    N, D, L = 64 * 8, 8, 64
+    q = np.repeat(rng.normal(size=(N // 64, D)), 64, axis=0)
+    k, v = rng.normal(size=(N, D)), rng.normal(size=(N, D))
+    r = orc.route(q, k, 64, L, 0.5)
+    a = orc.solattn_blocks(q, k, v, 64, L, 0.5, routing=r, order=1)
+    b = orc.solattn_blocks(q, k, v, 64, L, 0.5, routing=r, order=1, pooled_query_term=True)
+    assert np.allclose(a, b, rtol=0, atol=1e-14)
+    assert not np.allclose(a, orc.solattn_blocks(q, k, v, 64, L, 0.5, routing=r), atol=1e-6)
+
+
+def test_taylor_first_order_matches_brute_force_expansion():
+    # solattn_blocks(order=1) against a plain-loop evaluation of the expanded
+    # terms, block by block and row by row.
+    rng = np.random.default_rng(14)
+    N, D, L, tau = 64 * 6, 4, 64, 0.7
+    q, k, v = (rng.normal(size=(N, D)) for _ in range(3))
+    s = 1.0 / math.sqrt(D)
+    r = orc.route(q, k, 64, L, tau)
+    got = orc.solattn_blocks(q, k, v, 64, L, tau, routing=r, order=1)
+    M = N // 64
+    for i in range(M):
+        for rr in range(0, 64, 21):
+            row = q[64 * i + rr]
+            terms_w, terms_v = [], []
+            for j in range(M):
+                kb, vb = k[64 * j:64 * j + 64], v[64 * j:64 * j + 64]
+                if r.keep[i, j]:
+                    for t in range(64):
+                        terms_w.append(math.exp(s * sum(row[d] * kb[t, d] for d in range(D))))
+                        terms_v.append(vb[t])
+                else:
+                    km = [sum(kb[t, d] for t in range(64)) / 64 for d in range(D)]
+                    vm = [sum(vb[t, d] for t in range(64)) / 64 for d in range(D)]
+                    cov = [[sum((kb[t, a] - km[a]) * (vb[t, b] - vm[b]) for t in range(64)) / 64
+                            for b in range(D)] for a in range(D)]
+                    terms_w.append(64 * math.exp(s * sum(row[d] * km[d] for d in range(D))))
+                    terms_v.append(np.array([vm[b] + s * sum(row[a] * cov[a][b] for a in range(D))
+                                             for b in range(D)]))
+            want = sum(w * x for w, x in zip(terms_w, terms_v)) / sum(terms_w)
+            assert np.allclose(got[64 * i + rr], want, rtol=0, atol=1e-12)
