@@ -26,3 +26,20 @@ def test_reference_arm_json_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # a step is the bounded sample itself; the full-operator time is reported apart
+    assert d["ms_per_step"] < 60_000 < d["extrapolated_full_operator_ms"]
+    assert cb["cpu_model"]
+
+
+def test_cpu_baseline_times_routing_and_dense_oracle():
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_threshold_b200 import synthetic as syn
+    w = syn.workload("tiny_n1024")
+    o = bench.oracle_sample_rate(w, 1.0, 0.3, dense_budget_s=0.3)
+    assert o["route_s_per_head"] > 0 and o["blocks"] > 0 and o["dense_blocks"] > 0
+    assert o["rate"] > 0 and o["dense_rate"] > 0
+    # the extrapolation charges the routing of every head
+    per_block = o["seconds"] * o["cores"] / o["blocks"]
+    want = w.B * w.H * (o["route_s_per_head"] + w.M * per_block) / o["cores"]
+    assert abs(o["full_s"] - want) <= 1e-9 * want
