@@ -660,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       Stage s;
       int n = 0;
       bool ok = true;
+      uint32_t k_issued[kRingStages] = {}, v_issued[kRingStages] = {};
       while (ok && it.next(s, mU, mA, mB, M, P, no_corr)) {
         const int slot = n % kRingStages;
         const uint32_t use_parity = ((n / kRingStages) - 1) & 1;
@@ -674,6 +675,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(sK + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmKb : &tmK,
                         &bars[kBarKFull + slot], c * 64, row);
+          ++k_issued[slot];
         }
         if (n >= kRingStages)
           ok = mbar_wait(&bars[kBarVEmpty + slot], use_parity, abort_flag, err, 2, p.timeout_ns);
@@ -683,12 +685,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int c = 0; c < kChunks; ++c)
           tma_load_2d(sV + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmVb : &tmV,
                       &bars[kBarVFull + slot], c * 64, row);
+        ++v_issued[slot];
         ++n;
       }
       if (!ok || *abort_flag) {
-        // Let loads already issued land before the CTA's shared memory is released.
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 2000000ull) {
+        // Let the loads already issued land before the CTA's shared memory is
+        // released: the k-th load into a ring slot completes phase k - 1 of
+        // its full barrier (bounded waits that ignore the abort flag).
+        for (int i = 0; i < kRingStages; ++i) {
+          if (k_issued[i] > 0) mbar_wait_drain(&bars[kBarKFull + i], (k_issued[i] - 1) & 1, p.timeout_ns);
+          if (v_issued[i] > 0) mbar_wait_drain(&bars[kBarVFull + i], (v_issued[i] - 1) & 1, p.timeout_ns);
         }
       }
     }
@@ -749,10 +755,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mma_commit(&bars[kBarOFull]);
       mma_commit(&bars[kBarDrain]);
       // Drain: the CTA must not free TMEM while MMAs are still running.
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait_sleep(&bars[kBarDrain], 0, kWaitHintNs) &&
-             global_timer_ns() - t0 < 2000000000ull) {
-      }
+      mbar_wait_drain(&bars[kBarDrain], 0, 2000000000ull);
+      // A Q tile whose wait gave up must still land before shared memory is released.
+      if (!ok) mbar_wait_drain(&bars[kBarQ], 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue

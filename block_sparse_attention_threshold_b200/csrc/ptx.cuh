@@ -105,6 +105,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait used while a CTA drains after a give-up: the abort flag is ignored
+// (it is already raised), only the time limit ends the wait.  Returns
+// whether the phase completed.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 <= timeout_ns)
+    if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+  return false;
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2D tiled bulk-tensor load global -> shared, completion counted in bytes on
