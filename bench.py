@@ -476,6 +476,9 @@ def run_sweep(args):
     peaks = measured_peaks()
     for name in names:
         w = syn.workload(name)
+        if args.fp8:
+            run_sweep_fp8(args, w, dev, peaks)
+            continue
         qb, kb, vb = syn.generate_bf16(w)
         q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (qb, kb, vb))
         del qb, kb, vb
@@ -548,6 +551,68 @@ def run_sweep(args):
             print(json.dumps(row), flush=True)
         del q, k, v, out, ws
         torch.cuda.empty_cache()
+
+
+def run_sweep_fp8(args, w, dev, peaks):
+    """The 8-bit entry point on workload `w`: E4M3 inputs (scale 1), pooling
+    and attention timed alone with CUDA events (medians), one JSON line per tau.
+    The roofline denominator is twice the measured bf16 burst peak (the nominal
+    E4M3 / bf16 tensor-rate ratio), stated in the line."""
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_threshold_b200 import abi, synthetic as syn
+
+    bits = syn.generate_e4m3(w)
+    q8, k8, v8 = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in bits)
+    del bits
+    out = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+    nbytes, _ = abi.workspace_layout(w.B, w.H, w.N, w.D)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    pool_ms = timed(lambda: abi.pool_fp8(q8, k8, v8, ws), max(5, args.reps))
+    total = w.B * w.H * w.M * w.M
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    taus = [args.tau] if args.tau is not None else list(w.taus)
+    for tau in taus:
+        opts = abi.Opts()
+        cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+        opts.kept_pairs = cnt.data_ptr()
+        opts.exact_pairs = cnt.data_ptr() + 8
+        abi.attend_fp8(q8, k8, v8, ws, tau, w.prefix_len, out=out, opts=opts)
+        torch.cuda.synchronize()
+        kept, exact = (int(x) for x in cnt.cpu().tolist())
+        with ClockSampler(0) as clk:
+            att_ms = timed(lambda: abi.attend_fp8(q8, k8, v8, ws, tau, w.prefix_len, out=out), max(5, args.reps))
+        kept_fl = kept * 4.0 * 64 * 64 * w.D
+        corr_fl = (total - kept) * 4.0 * 64 * w.D
+        step = pool_ms + att_ms
+        row = {
+            "workload": w.name, "tau": tau, "precision": "e4m3 inputs, e4m3 P, fp32 accumulate, bf16 out",
+            "kept_frac": kept / total, "exact_frac": exact / total,
+            "attend_ms": att_ms, "pool_ms": pool_ms,
+            "dense_equiv_tflops": w.dense_flops() / step / 1e9,
+            "actual_tflops_kept_plus_corr": (kept_fl + corr_fl) / att_ms / 1e9,
+            "fp8_peak_tflops": fp8_peak,
+            "frac_of_fp8_peak": (kept_fl + corr_fl) / att_ms / 1e9 / fp8_peak,
+            "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal E4M3/bf16 ratio)",
+            "pool_gbs": (3.0 * w.B * w.H * w.N * w.D + w.B * w.H * w.M * w.D * 10) / pool_ms / 1e6,
+            "device_status": abi.device_status(),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(row), flush=True)
 
 
 def run_prep(args):
@@ -671,6 +736,8 @@ def main():
     ap.add_argument("--rope-dims", type=int, default=None, help="--prep: rotated dimensions (default D/2)")
     ap.add_argument("--sweep-min-ms", type=float, default=500.0,
                     help="--sweep: lower bound on each attend timing region (more launches if needed)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="--sweep with the 8-bit entry point (E4M3 inputs); frac against twice the bf16 peak")
     ap.add_argument("--budget-sparsity", type=float, default=None,
                     help="--sweep with fixed-budget routing keeping (1 - s) of the video blocks, "
                          "skipped blocks dropped (the draft stage's block-sparse attention)")

@@ -60,6 +60,9 @@ _SIGS = {
     "sol_attn_pool": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "sol_attn_attend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(Opts), _P]),
     "sol_attn_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "sol_attn_forward_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _F, _F, _F, ctypes.POINTER(Opts), _P]),
+    "sol_attn_pool_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P]),
+    "sol_attn_attend_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _F, _F, _F, ctypes.POINTER(Opts), _P]),
     "sol_attn_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
     "sol_attn_qknorm_rope_pool": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
     "sol_attn_device_status": (_I, [_P]),
@@ -153,6 +156,56 @@ def forward_noalloc(q, k, v, tau: float, prefix_len: int = 0, out=None, stream=N
                                         B, H, N, D, block, float(tau), int(prefix_len),
                                         _stream(stream))
     _check(st, "sol_attn_forward_noalloc")
+    return out
+
+
+def forward_fp8(q8, k8, v8, tau: float, prefix_len: int = 0, q_scale: float = 1.0, k_scale: float = 1.0,
+                v_scale: float = 1.0, out=None, opts: Opts | None = None, stream=None, block: int = BLOCK):
+    """Sol-Attn on E4M3 inputs through sol_attn_forward_fp8.  q8, k8, v8 are
+    CUDA uint8 tensors [B, H, N, D] holding E4M3 bytes (real value = decoded
+    byte times the tensor's scale); returns the bf16 output."""
+    import torch
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA uint8 tensor of E4M3 bytes")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, D]")
+    if not (q8.shape == k8.shape == v8.shape):
+        raise ValueError("q8, k8, v8 must have the same shape")
+    B, H, N, D = (int(x) for x in q8.shape)
+    if out is None:
+        out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    elif out.shape != q8.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q8")
+    st = lib().sol_attn_forward_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                                    B, H, N, D, block, float(tau), int(prefix_len), float(q_scale),
+                                    float(k_scale), float(v_scale),
+                                    ctypes.byref(opts) if opts is not None else None, _stream(stream))
+    _check(st, "sol_attn_forward_fp8")
+    return out
+
+
+def pool_fp8(q8, k8, v8, workspace, q_scale: float = 1.0, k_scale: float = 1.0, stream=None) -> None:
+    """Pooling of E4M3 inputs into `workspace` (CUDA uint8) via sol_attn_pool_fp8."""
+    B, H, N, D = (int(x) for x in q8.shape)
+    st = lib().sol_attn_pool_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), workspace.data_ptr(),
+                                 B, H, N, D, float(q_scale), float(k_scale), _stream(stream))
+    _check(st, "sol_attn_pool_fp8")
+
+
+def attend_fp8(q8, k8, v8, workspace, tau: float, prefix_len: int = 0, q_scale: float = 1.0,
+               k_scale: float = 1.0, v_scale: float = 1.0, out=None, opts: Opts | None = None, stream=None,
+               block: int = BLOCK):
+    """Routing + attention on a pool_fp8 workspace via sol_attn_attend_fp8."""
+    import torch
+    B, H, N, D = (int(x) for x in q8.shape)
+    if out is None:
+        out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    st = lib().sol_attn_attend_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                                   workspace.data_ptr(), B, H, N, D, block, float(tau), int(prefix_len),
+                                   float(q_scale), float(k_scale), float(v_scale),
+                                   ctypes.byref(opts) if opts is not None else None, _stream(stream))
+    _check(st, "sol_attn_attend_fp8")
     return out
 
 

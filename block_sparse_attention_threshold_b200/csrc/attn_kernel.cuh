@@ -85,15 +85,18 @@ struct AttnParams {
   int skip_first_k_arrival;  // test hook: producer never loads stage 0
   int budget;                // > 0: keep this many top-scoring video blocks per query block
   bool correct;              // pooled correction of skipped blocks (else they are dropped)
+  float out_scale;           // O is multiplied by this (the value scale of 8-bit V; 1 otherwise)
 };
 
-template <int D>
+// kElem: bytes per element, 2 (bf16) or 1 (E4M3).  Tiles are stored in
+// 128-byte column chunks (64 bf16 or 128 E4M3 values) with 128-byte swizzle.
+template <int D, int kElem = 2>
 struct SmemPlan {
-  static constexpr int kBlockBytes = kStageKeys * D * 2;  // one 64-key block of K (or V)
-  static constexpr int kChunkBytes = kStageKeys * 128;    // its 64-column chunk (8 KB)
-  static constexpr int kQChunkBytes = kTileM * 128;       // 64-column chunk of the Q tile
+  static constexpr int kBlockBytes = kStageKeys * D * kElem;  // one 64-key block of K (or V)
+  static constexpr int kChunkBytes = kStageKeys * 128;        // its 128-byte column chunk (8 KB)
+  static constexpr int kQChunkBytes = kTileM * 128;           // 128-byte column chunk of the Q tile
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileM * D * 2;           // K ring
+  static constexpr int kK = kQ + kTileM * D * kElem;           // K ring
   static constexpr int kV = kK + kRingStages * kBlockBytes;  // V ring
   static constexpr int kMaskA = kV + kRingStages * kBlockBytes;
   static constexpr int kMaskB = kMaskA + kMaskWords * 4;
@@ -273,11 +276,11 @@ __device__ __forceinline__ uint32_t score_key(float x) {
 // The cut is found exactly by a 4-pass, 8-bit radix select over the score
 // keys (shared-memory histograms, one warp picks each digit); a single warp
 // then writes the keep words in block order, which settles ties.
-template <int D>
+template <int D, int kElem>
 __device__ __forceinline__ void route_budget_masks(const AttnParams& p, const float* sc, uint8_t* smem,
                                                    int tid, bool videoA, bool videoB, bool hasB,
                                                    uint32_t* mA, uint32_t* mB) {
-  using L = SmemPlan<D>;
+  using L = SmemPlan<D, kElem>;
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L::kHist);  // [2][256]
   uint32_t* bc = hist + 512;                                      // broadcast words
   const int M = p.M, P = p.P, nv = M - P;
@@ -378,10 +381,10 @@ __device__ __forceinline__ void route_budget_masks(const AttnParams& p, const fl
 // Router: pooled scores of query blocks iA, iB against every video key
 // block, population mean/std, threshold, keep bits.  Runs on all the CTA's
 // threads before the mainloop; scores live in the (not yet used) K/V rings.
-template <int D>
+template <int D, int kElem>
 __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, int iB, bool hasB,
                                            uint8_t* smem, int tid, float pre_a, float pre_b) {
-  using L = SmemPlan<D>;
+  using L = SmemPlan<D, kElem>;
   uint32_t* mA = reinterpret_cast<uint32_t*>(smem + L::kMaskA);
   uint32_t* mB = reinterpret_cast<uint32_t*>(smem + L::kMaskB);
   float* sq = reinterpret_cast<float*>(smem + L::kQbar);
@@ -462,7 +465,7 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
     }
     __syncthreads();
     if (p.budget > 0) {
-      route_budget_masks<D>(p, sc, smem, tid, videoA, videoB, hasB, mA, mB);
+      route_budget_masks<D, kElem>(p, sc, smem, tid, videoA, videoB, hasB, mA, mB);
       return;
     }
     // Pass 1: mean (and exact-equality check through min/max).
@@ -521,15 +524,21 @@ __device__ __forceinline__ void route_tile(const AttnParams& p, int bh, int iA, 
   }
 }
 
-template <int D, bool kDense>
+template <int D, bool kDense, bool kFp8 = false>
 __global__ void __launch_bounds__(kThreads, 2)
     sol_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmKb,
                         const __grid_constant__ CUtensorMap tmVb, const AttnParams p) {
-  using L = SmemPlan<D>;
-  constexpr int kChunks = D / 64;
+  // kFp8: E4M3 Q, K, V and pooled K/V, tcgen05.mma kind::f8f6f4 (32 values of K
+  // per instruction), P stored to TMEM as E4M3, four per column.
+  constexpr int kElem = kFp8 ? 1 : 2;
+  using L = SmemPlan<D, kElem>;
+  constexpr int kChunks = D * kElem / 128;
+  constexpr int kChunkElems = 128 / kElem;   // values per 128-byte chunk row
+  constexpr int kMmaK = 32 / kElem;          // K of one MMA instruction
+  static_assert(!kFp8 || D == 128, "the 8-bit path is built for D = 128");
   constexpr uint32_t kTmemCols = 256;
   constexpr uint32_t kColO = 128;  // S buffer b at columns [64 b, 64 b + 64)
 
@@ -612,12 +621,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     const size_t row0 = static_cast<size_t>(bh) * p.N + static_cast<size_t>(qt) * kTileM;
-    mbar_arrive_expect_tx(&bars[kBarQ], kTileM * D * 2);
+    mbar_arrive_expect_tx(&bars[kBarQ], kTileM * D * kElem);
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int c = 0; c < kChunks; ++c)
-        tma_load_2d(sQ + c * L::kQChunkBytes + h * 64 * 128, &tmQ, &bars[kBarQ], c * 64,
+        tma_load_2d(sQ + c * L::kQChunkBytes + h * 64 * 128, &tmQ, &bars[kBarQ], c * kChunkElems,
                     static_cast<int>(row0 + h * 64));
   }
 
@@ -631,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mB[w] = fullw;
     }
   } else {
-    route_tile<D>(p, bh, iA, iB, hasB, smem, tid, pre_qa, pre_qb);
+    route_tile<D, kElem>(p, bh, iA, iB, hasB, smem, tid, pre_qa, pre_qb);
   }
   __syncthreads();
   for (int w = tid; w < nw; w += kThreads) mU[w] = mA[w] | mB[w];
@@ -674,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(sK + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmKb : &tmK,
-                        &bars[kBarKFull + slot], c * 64, row);
+                        &bars[kBarKFull + slot], c * kChunkElems, row);
           ++k_issued[slot];
         }
         if (n >= kRingStages)
@@ -684,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int c = 0; c < kChunks; ++c)
           tma_load_2d(sV + slot * L::kBlockBytes + c * L::kChunkBytes, s.corr ? &tmVb : &tmV,
-                      &bars[kBarVFull + slot], c * 64, row);
+                      &bars[kBarVFull + slot], c * kChunkElems, row);
         ++v_issued[slot];
         ++n;
       }
@@ -708,8 +717,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t vdesc = sdesc_sw128(smem_u32(sV), L::kChunkBytes, 1024);
-      const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kStageKeys, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, true);
+      const uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32(kTileM, kStageKeys, false)
+                                     : idesc_bf16_f32(kTileM, kStageKeys, false);
+      const uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(kTileM, D, true) : idesc_bf16_f32(kTileM, D, true);
       const int total = count_stages(mU, mA, mB, M, P, no_corr);
       bool ok = mbar_wait(&bars[kBarQ], 0, abort_flag, err, 3, p.timeout_ns);
       // S(n) = Q K(n)^T into S buffer n % 2; A = Q (K-major SW128), B = K.
@@ -721,10 +731,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint64_t kd = kdesc + static_cast<uint32_t>((slot * L::kBlockBytes) >> 4);
         const uint32_t dcol = tmem + 64u * (n & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / kMmaK; ++kk) {
+          // 32 bytes of K per instruction: four steps per 128-byte chunk.
           constexpr int kQStep = L::kQChunkBytes >> 4, kKStep = L::kChunkBytes >> 4;
-          mma_bf16_ss(dcol, qdesc + static_cast<uint32_t>((kk >> 2) * kQStep + (kk & 3) * 2),
-                      kd + static_cast<uint32_t>((kk >> 2) * kKStep + (kk & 3) * 2), idesc_qk, kk > 0);
+          const uint64_t ad = qdesc + static_cast<uint32_t>((kk >> 2) * kQStep + (kk & 3) * 2);
+          const uint64_t bd = kd + static_cast<uint32_t>((kk >> 2) * kKStep + (kk & 3) * 2);
+          if constexpr (kFp8)
+            mma_e4m3_ss(dcol, ad, bd, idesc_qk, kk > 0);
+          else
+            mma_bf16_ss(dcol, ad, bd, idesc_qk, kk > 0);
         }
         mma_commit(&bars[kBarSFull + (n & 1)]);
         mma_commit(&bars[kBarKEmpty + slot]);
@@ -742,9 +757,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t pcol = tmem + 64u * (n & 1);
         const uint64_t vd = vdesc + static_cast<uint32_t>((slot * L::kBlockBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kStageKeys / 16; ++kk) {
-          mma_bf16_ts(tmem + kColO, pcol + kk * 8, vd + static_cast<uint32_t>(kk * ((16 * 128) >> 4)),
-                      idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kStageKeys / kMmaK; ++kk) {
+          // kMmaK keys per instruction: 32 bytes of P (8 TMEM columns) and
+          // kMmaK 128-byte rows of V.
+          const uint64_t bd = vd + static_cast<uint32_t>(kk * ((kMmaK * 128) >> 4));
+          if constexpr (kFp8)
+            mma_e4m3_ts(tmem + kColO, pcol + kk * 8, bd, idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_bf16_ts(tmem + kColO, pcol + kk * 8, bd, idesc_pv, (n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars[kBarVEmpty + slot]);
         mma_commit(&bars[kBarOReady]);
@@ -787,6 +807,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         use1 = v1 ? (~rowmask[(lo >> 5) + 1] & v1) : 0u;
       }
       uint32_t pk0[16], pk1[16];
+      float ea0 = 0.f, ea1 = 0.f, eb0 = 0.f, eb1 = 0.f;  // E4M3 path: the even pair of a column
       float alpha = 1.0f;
       bool warp_need = false;
       if (__any_sync(0xFFFFFFFFu, (use0 | use1) != 0u)) {
@@ -855,8 +876,17 @@ __global__ void __launch_bounds__(kThreads, 2)
               acc0 = f2_add(acc0, pa);
               acc2 = f2_add(acc2, pb);
             }
-            pk0[c] = pack_bf16x2(a0, a1);
-            pk1[c] = pack_bf16x2(b0, b1);
+            if constexpr (kFp8) {
+              if (c & 1) {
+                pk0[c >> 1] = pack_e4m3x4(ea0, ea1, a0, a1);
+                pk1[c >> 1] = pack_e4m3x4(eb0, eb1, b0, b1);
+              } else {
+                ea0 = a0; ea1 = a1; eb0 = b0; eb1 = b1;
+              }
+            } else {
+              pk0[c] = pack_bf16x2(a0, a1);
+              pk1[c] = pack_bf16x2(b0, b1);
+            }
           }
         } else {
 #pragma unroll
@@ -880,8 +910,17 @@ __global__ void __launch_bounds__(kThreads, 2)
               acc0 = f2_add(acc0, pa);
               acc2 = f2_add(acc2, pb);
             }
-            pk0[c] = pack_bf16x2(a0, a1);
-            pk1[c] = pack_bf16x2(b0, b1);
+            if constexpr (kFp8) {
+              if (c & 1) {
+                pk0[c >> 1] = pack_e4m3x4(ea0, ea1, a0, a1);
+                pk1[c >> 1] = pack_e4m3x4(eb0, eb1, b0, b1);
+              } else {
+                ea0 = a0; ea1 = a1; eb0 = b0; eb1 = b1;
+              }
+            } else {
+              pk0[c] = pack_bf16x2(a0, a1);
+              pk1[c] = pack_bf16x2(b0, b1);
+            }
           }
         }
         const uint64_t a = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
@@ -895,8 +934,19 @@ __global__ void __launch_bounds__(kThreads, 2)
           pk1[c] = 0u;
         }
       }
-      tmem_st16(scol + 0, pk0);
-      tmem_st16(scol + 16, pk1);
+      if constexpr (kFp8) {
+        // 64 keys of E4M3 P: columns 0-7 from the first 32 keys, 8-15 from the rest.
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pk[i] = pk0[i];
+          pk[8 + i] = pk1[i];
+        }
+        tmem_st16(scol + 0, pk);
+      } else {
+        tmem_st16(scol + 0, pk0);
+        tmem_st16(scol + 16, pk1);
+      }
       // Every stage n >= 1 waits for PV(n-1) (the n-th commit on OReady).
       // Waiting each time keeps the parity unambiguous: PV(n-2) is known to
       // be done, so only phase n-1 can be pending.  The wait sits after this
@@ -929,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok) ok = mbar_wait(&bars[kBarOFull], 0, abort_flag, err, 8, p.timeout_ns);
     if (ok) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+      const float inv_l = l > 0.f ? p.out_scale / l : 0.f;
       const int grow = qt * kTileM + r;
       __nv_bfloat16* dst = p.out + (static_cast<size_t>(bh) * p.N + grow) * D;
 #pragma unroll

@@ -62,6 +62,9 @@ int check_device() {
     ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<64, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                sol::SmemPlan<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(sol::sol_attn_fwd_kernel<128, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sol::SmemPlan<128, 1>::kAlloc) == cudaSuccess;
     c.status = ok ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
   });
   return c.status;
@@ -92,6 +95,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2D view [rows, D] of an 8-bit array (E4M3 bytes), 64-row x 128-byte boxes,
+// 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D)};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -195,6 +213,7 @@ int launch_attend(const void* q, const void* k, const void* v, void* out, const 
   p.skip_first_k_arrival = o ? o->test_skip_first_k_load : 0;
   p.budget = o ? o->budget_blocks : 0;
   p.correct = !(o != nullptr && o->skip_correction != 0);
+  p.out_scale = 1.0f;
 
   const long long tiles = static_cast<long long>(B) * H * p.tiles_per_head;
   dim3 grid(static_cast<unsigned>(tiles));
@@ -484,6 +503,131 @@ const char* sol_attn_status_string(int status) {
     case SOL_ATTN_ERR_DEVICE_TIMEOUT: return "SOL_ATTN_ERR_DEVICE_TIMEOUT";
     default: return "SOL_ATTN_ERR_UNKNOWN";
   }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// 8-bit (E4M3) forward: the same operator on E4M3 inputs with per-tensor
+// scales, the exact-block and correction products on kind::f8f6f4 tensor
+// cores, P rounded to E4M3.
+namespace {
+
+int launch_attend_e4m3(const void* q, const void* k, const void* v, void* out, const Workspace& w, int B,
+                       int H, int N, float tau, int prefix_len, float q_scale, float k_scale, float v_scale,
+                       const sol_attn_opts* o, cudaStream_t s) {
+  constexpr int D = 128;
+  const int M = N / SOL_ATTN_BLOCK;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
+  const uint64_t prows = static_cast<uint64_t>(B) * H * M;
+  CUtensorMap mq, mk, mv, mkb, mvb;
+  if (!make_map_u8(&mq, q, rows, D) || !make_map_u8(&mk, k, rows, D) || !make_map_u8(&mv, v, rows, D) ||
+      !make_map_u8(&mkb, w.kbar_bf16, prows, D) || !make_map_u8(&mvb, w.vbar_bf16, prows, D))
+    return SOL_ATTN_ERR_CUDA;
+  sol::AttnParams p{};
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.M = M;
+  p.P = prefix_len / SOL_ATTN_BLOCK;
+  p.tiles_per_head = (M + 1) / 2;
+  p.tau = tau;
+  const float scale = (o != nullptr && o->softmax_scale > 0.f) ? o->softmax_scale : 1.0f / std::sqrt(128.0f);
+  p.scale = scale;                                               // router: real-domain pooled values
+  p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;  // logits of raw E4M3 products
+  p.out_scale = v_scale;
+  p.qbar = w.qbar;
+  p.kbar = w.kbar;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.debug_mask = o ? o->debug_mask : nullptr;
+  p.kept_pairs = o ? o->kept_pairs : nullptr;
+  p.exact_pairs = o ? o->exact_pairs : nullptr;
+  const unsigned tms = (o != nullptr && o->timeout_ms > 0) ? o->timeout_ms : 1000u;
+  p.timeout_ns = static_cast<uint64_t>(tms) * 1000000ull;
+  p.skip_first_k_arrival = o ? o->test_skip_first_k_load : 0;
+  p.budget = o ? o->budget_blocks : 0;
+  p.correct = !(o != nullptr && o->skip_correction != 0);
+  const long long tiles = static_cast<long long>(B) * H * p.tiles_per_head;
+  sol::sol_attn_fwd_kernel<128, false, true><<<dim3(static_cast<unsigned>(tiles)), sol::kThreads,
+                                               sol::SmemPlan<128, 1>::kAlloc, s>>>(mq, mk, mv, mkb, mvb, p);
+  return cudaGetLastError() == cudaSuccess ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+}
+
+bool good_scale(float x) { return std::isfinite(x) && x > 0.f; }
+
+int check_scales(float q_scale, float k_scale, float v_scale) {
+  return good_scale(q_scale) && good_scale(k_scale) && good_scale(v_scale) ? SOL_ATTN_OK : SOL_ATTN_ERR_INVALID_ARG;
+}
+
+int launch_pool_e4m3(const void* q, const void* k, const void* v, const Workspace& w, int B, int H, int N,
+                     float q_scale, float k_scale, cudaStream_t s) {
+  const unsigned nblk = static_cast<unsigned>(static_cast<long long>(B) * H * (N / SOL_ATTN_BLOCK));
+  sol::PoolOutE4M3 po{w.qbar, w.kbar, reinterpret_cast<uint8_t*>(w.kbar_bf16),
+                      reinterpret_cast<uint8_t*>(w.vbar_bf16), q_scale, k_scale};
+  sol::pool_kernel_e4m3<128><<<dim3(nblk, 3), 128, 0, s>>>(static_cast<const uint8_t*>(q),
+                                                          static_cast<const uint8_t*>(k),
+                                                          static_cast<const uint8_t*>(v), po);
+  return cudaGetLastError() == cudaSuccess ? SOL_ATTN_OK : SOL_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sol_attn_pool_fp8(const void* q, const void* k, const void* v, void* workspace, int B, int H, int N, int D,
+                      float q_scale, float k_scale, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return SOL_ATTN_OK;
+  if (st != SOL_ATTN_OK) return st;
+  if (D != 128) return SOL_ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !workspace || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_scales(q_scale, k_scale, 1.0f)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  return launch_pool_e4m3(q, k, v, split_workspace(workspace, B, H, N, D), B, H, N, q_scale, k_scale,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_attend_fp8(const void* q, const void* k, const void* v, void* out, const void* workspace, int B,
+                        int H, int N, int D, int block, float tau, int prefix_len, float q_scale, float k_scale,
+                        float v_scale, const sol_attn_opts* opts, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if (D != 128) return SOL_ATTN_ERR_UNSUPPORTED;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SOL_ATTN_ERR_INVALID_ARG;
+  if ((st = check_scales(q_scale, k_scale, v_scale)) != SOL_ATTN_OK) return st;
+  if ((st = check_opts(opts)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  return launch_attend_e4m3(q, k, v, out, split_workspace(workspace, B, H, N, D), B, H, N, tau, prefix_len,
+                            q_scale, k_scale, v_scale, opts, static_cast<cudaStream_t>(stream));
+}
+
+int sol_attn_forward_fp8(const void* q, const void* k, const void* v, void* out, int B, int H, int N, int D,
+                         int block, float tau, int prefix_len, float q_scale, float k_scale, float v_scale,
+                         const sol_attn_opts* opts, void* stream) {
+  int st = check_shape(B, H, N, D);
+  if (st == -1) return check_route_args(block, tau, prefix_len, N);
+  if (st != SOL_ATTN_OK) return st;
+  if (D != 128) return SOL_ATTN_ERR_UNSUPPORTED;
+  if ((st = check_route_args(block, tau, prefix_len, N)) != SOL_ATTN_OK) return st;
+  if ((st = check_io(q, k, v, out)) != SOL_ATTN_OK) return st;
+  if ((st = check_scales(q_scale, k_scale, v_scale)) != SOL_ATTN_OK) return st;
+  if ((st = check_opts(opts)) != SOL_ATTN_OK) return st;
+  if ((st = check_device()) != SOL_ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = sol_attn_workspace_bytes(B, H, N, D, nullptr);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return SOL_ATTN_ERR_CUDA;
+  const Workspace w = split_workspace(ws, B, H, N, D);
+  st = launch_pool_e4m3(q, k, v, w, B, H, N, q_scale, k_scale, s);
+  if (st == SOL_ATTN_OK)
+    st = launch_attend_e4m3(q, k, v, out, w, B, H, N, tau, prefix_len, q_scale, k_scale, v_scale, opts, s);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == SOL_ATTN_OK) st = SOL_ATTN_ERR_CUDA;
+  return st;
 }
 
 }  // extern "C"

@@ -142,6 +142,46 @@ def bf16_bits_to_fp64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
+E4M3_MAX = 448.0  # largest finite OCP FP8 E4M3 value, 1.75 * 2^8
+
+
+def fp64_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 to OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3
+    mantissa bits; no infinities) with round-to-nearest-even in one step,
+    saturating at +-448; returns uint8 bits.
+
+    A value's quantum is 2^(e - 3) for its binade exponent e, with e taken as
+    at least -6 so that the subnormals (quantum 2^-9) share the smallest
+    normal binade's spacing.  x / quantum is exact in fp64, so rounding it
+    with numpy's rint (ties to even) is exact RNE.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    neg = np.signbit(x)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    _, ex = np.frexp(a)                       # a = m * 2^ex, m in [0.5, 1)
+    e = np.clip(ex - 1, -6, 8)
+    q = np.ldexp(1.0, (e - 3).astype(np.int64))
+    r = np.rint(a / q) * q                    # representable; may step up one binade
+    _, er = np.frexp(r)
+    er = er - 1
+    normal = r >= 2.0 ** -6
+    exp_field = np.where(normal, er + 7, 0)
+    mant = np.where(normal, np.rint(np.ldexp(r, -er.astype(np.int64)) * 8) - 8, np.rint(r * 2.0 ** 9))
+    bits = (exp_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    bits = np.where(neg, bits | 0x80, bits)
+    return bits.astype(np.uint8)
+
+
+def e4m3_bits_to_fp64(bits: np.ndarray) -> np.ndarray:
+    """Decode E4M3 bits (uint8) exactly; the two NaN codes (S.1111.111) give NaN."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    e = (b >> 3) & 15
+    m = b & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, np.ldexp(8.0 + m, (e - 10).astype(np.int64)))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(b & 0x80, -mag, mag)
+
+
 def _heads(w: Workload, rng: np.random.Generator) -> Iterator[tuple]:
     """Yield (b, h, q64, k64, v64) in draw order, fp64 [N, D] each."""
     proj = rng.standard_normal((w.H, EMB_DIM, w.D)) / math.sqrt(w.D)
@@ -168,6 +208,23 @@ def generate_bf16(w: Workload) -> tuple:
         q[b, h] = fp64_to_bf16_bits(q64)
         k[b, h] = fp64_to_bf16_bits(k64)
         v[b, h] = fp64_to_bf16_bits(v64)
+    return q, k, v
+
+
+def generate_e4m3(w: Workload, scales=(1.0, 1.0, 1.0)) -> tuple:
+    """Q, K, V as E4M3 bits, uint8 [B, H, N, D] each: the same draws as
+    generate_bf16, each value divided by its tensor's scale and rounded once
+    from fp64 to E4M3 (the real value is then the decoded byte times the
+    scale)."""
+    shape = (w.B, w.H, w.N, w.D)
+    q = np.empty(shape, np.uint8)
+    k = np.empty(shape, np.uint8)
+    v = np.empty(shape, np.uint8)
+    sq, sk, sv = (float(x) for x in scales)
+    for b, h, q64, k64, v64 in _heads(w, np.random.default_rng(w.seed)):
+        q[b, h] = fp64_to_e4m3_bits(q64 / sq)
+        k[b, h] = fp64_to_e4m3_bits(k64 / sk)
+        v[b, h] = fp64_to_e4m3_bits(v64 / sv)
     return q, k, v
 
 

@@ -24,6 +24,9 @@
  *       (count-weighted mean-key logit + ln c_j, mean value).
  *  [R6] [R3]'s page, same section, fused-operators item: the QKNorm +
  *       partial RoPE chain keeps its intermediates in registers or on chip.
+ *  [R7] [R1]'s page, section "latent hand-off: 384p draft to 768p refine":
+ *       the DiT runs with 8-bit (W8A8 FP8) weights and activations; [R3]'s
+ *       page, same section, multi-GPU item: attention outputs travel as FP8.
  *
  * Conventions shared by every entry point
  *  - q, k, v, out: DEVICE pointers to contiguous bf16 arrays laid out
@@ -177,6 +180,38 @@ int sol_attn_attend(const void* q, const void* k, const void* v, void* out,
 int sol_attn_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B,
                              int H, int N, int D, int block, float tau, int prefix_len,
                              void* stream);
+
+/* 8-bit variant of sol_attn_forward_ex [R1]-[R4], [R7]: q, k, v are DEVICE
+ * arrays of E4M3 bytes (OCP FP8 E4M3: 1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, largest finite 448), laid out [B][H][N][D] like the bf16
+ * inputs, 16-byte aligned; the real values are the decoded bytes times
+ * q_scale, k_scale, v_scale (finite, > 0; INVALID_ARG otherwise).  out is
+ * bf16 [B][H][N][D] as elsewhere.  D must be 128 (UNSUPPORTED otherwise).
+ * The operator is the same as sol_attn_forward's on the real values:
+ *  - pooling and routing are computed in fp32 from the decoded values, so
+ *    the keep mask follows the same definition;
+ *  - the exact blocks and the pooled correction run on 8-bit tensor cores
+ *    (fp32 accumulation): the pooled means used there are rounded to E4M3,
+ *    and the probabilities P to E4M3 before the P V product.
+ * Those two roundings are the only differences from the bf16 path's
+ * arithmetic; the accuracy this gives is stated in the design notes.
+ * `opts` (may be NULL) as in sol_attn_forward_ex.  Scratch, streams and
+ * errors as in sol_attn_forward. */
+int sol_attn_forward_fp8(const void* q, const void* k, const void* v, void* out, int B, int H, int N,
+                         int D, int block, float tau, int prefix_len, float q_scale, float k_scale,
+                         float v_scale, const sol_attn_opts* opts, void* stream);
+
+/* sol_attn_forward_fp8's two steps alone, as sol_attn_pool / sol_attn_attend
+ * are sol_attn_forward's: pooling of the E4M3 inputs into `workspace`
+ * (sol_attn_workspace_bytes(B, H, N, 128) bytes, 256-byte aligned: the fp32
+ * means of the real values for routing, and E4M3 means of the raw values in
+ * the first half of the two 16-bit sections), then routing and attention on
+ * that workspace.  Same argument rules as sol_attn_forward_fp8. */
+int sol_attn_pool_fp8(const void* q, const void* k, const void* v, void* workspace, int B, int H, int N,
+                      int D, float q_scale, float k_scale, void* stream);
+int sol_attn_attend_fp8(const void* q, const void* k, const void* v, void* out, const void* workspace,
+                        int B, int H, int N, int D, int block, float tau, int prefix_len, float q_scale,
+                        float k_scale, float v_scale, const sol_attn_opts* opts, void* stream);
 
 /* Host-buffer variant of sol_attn_forward: q, k, v and out are HOST
  * pointers, same [B][H][N][D] bf16 layout and the same result.  The pages

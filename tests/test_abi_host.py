@@ -22,7 +22,7 @@ def L():
 
 def test_every_declared_symbol_is_exported(L):
     names = abi.declared_symbols(HEADER)
-    assert len(names) == 11
+    assert len(names) == 14
     out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -116,6 +116,23 @@ def test_argument_validation_happens_before_any_device_call(L):
     assert prep(ws=FAKE, v=0) == E.ERR_INVALID_ARG  # pooling needs v
     assert prep(D=96) == E.ERR_UNSUPPORTED
     assert prep(N=0) == E.OK
+    # 8-bit entry point: D = 128 only, positive finite scales
+    def fp8(D=128, qs=1.0, ks=1.0, vs=1.0, q=FAKE, tau=1.0, B=1):
+        return L.sol_attn_forward_fp8(q, FAKE, FAKE, FAKE * 2, B, 2, 128, D, 64, tau, 0, qs, ks, vs, None, None)
+    assert fp8(D=64) == E.ERR_UNSUPPORTED
+    assert fp8(D=96) == E.ERR_UNSUPPORTED
+    assert fp8(qs=0.0) == E.ERR_INVALID_ARG
+    assert fp8(ks=-1.0) == E.ERR_INVALID_ARG
+    assert fp8(vs=math.inf) == E.ERR_INVALID_ARG
+    assert fp8(qs=math.nan) == E.ERR_INVALID_ARG
+    assert fp8(q=FAKE + 8) == E.ERR_INVALID_ARG
+    assert fp8(tau=math.nan) == E.ERR_INVALID_ARG
+    assert fp8(B=0) == E.OK
+    assert L.sol_attn_pool_fp8(FAKE, FAKE, FAKE, FAKE + 16, 1, 1, 64, 128, 1.0, 1.0, None) == E.ERR_INVALID_ARG
+    assert L.sol_attn_pool_fp8(FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 64, 1.0, 1.0, None) == E.ERR_UNSUPPORTED
+    assert L.sol_attn_pool_fp8(FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 128, 0.0, 1.0, None) == E.ERR_INVALID_ARG
+    assert L.sol_attn_attend_fp8(FAKE, FAKE, FAKE, FAKE * 2, None, 1, 1, 64, 128, 64, 1.0, 0, 1.0, 1.0, 1.0,
+                                 None, None) == E.ERR_INVALID_ARG
 
 
 def test_python_binding_rejects_non_cuda_tensors(L):

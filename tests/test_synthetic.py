@@ -60,3 +60,49 @@ def test_sample_query_blocks():
     assert len(s) == 64 and len(set(s.tolist())) == 64
     assert {0, 16, 511} <= set(s.tolist())
     assert np.array_equal(syn.sample_query_blocks(10, 2, 64, 5), np.arange(10))
+
+
+# --------------------------------------------------------------------------- E4M3 inputs
+
+def test_e4m3_hand_values():
+    enc = syn.fp64_to_e4m3_bits
+    cases = {
+        1.0: 0x38, 2.0: 0x40, 0.5: 0x30, -1.0: 0xB8, 448.0: 0x7E, -448.0: 0xFE,
+        1e6: 0x7E,                 # saturates at the largest finite value
+        2.0 ** -6: 0x08,           # smallest normal
+        2.0 ** -9: 0x01,           # smallest subnormal
+        2.0 ** -10: 0x00,          # half of it: tie to even (zero)
+        3 * 2.0 ** -10: 0x02,      # between 1 and 2 quanta of 2^-9: tie to even (2)
+        1.0625: 0x38,              # between 1.0 and 1.125: tie to even (1.0)
+        1.1875: 0x3A,              # between 1.125 and 1.25: tie to even (1.25)
+        1.05: 0x38, 1.07: 0x39,    # ordinary rounding (1.07 is nearer 1.125)
+        240.0: 0x77, 232.0: 0x76,  # 232 = 7.25 * 32 ties to 224 (even), 240 = 1.875 * 2^7
+    }
+    for x, b in cases.items():
+        assert int(enc(np.array([x]))[0]) == b, (x, hex(int(enc(np.array([x]))[0])), hex(b))
+
+
+def test_e4m3_decode_and_round_trip_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = syn.e4m3_bits_to_fp64(codes)
+    finite = ~np.isnan(vals)
+    assert np.isnan(vals[0x7F]) and np.isnan(vals[0xFF]) and finite.sum() == 254
+    assert vals[0x7E] == 448.0 and vals[0x01] == 2.0 ** -9 and vals[0x38] == 1.0
+    # every finite code decodes and re-encodes to itself (0x80 is -0, which encodes back to 0x80)
+    back = syn.fp64_to_e4m3_bits(vals[finite])
+    assert np.array_equal(back, codes[finite])
+    # positive codes are increasing
+    pos = vals[0:0x7F]
+    assert np.all(np.diff(pos) > 0)
+
+
+def test_e4m3_rounding_is_nearest_on_random_values():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(20000) * rng.choice([1e-3, 0.1, 1.0, 30.0], size=20000)
+    got = syn.e4m3_bits_to_fp64(syn.fp64_to_e4m3_bits(x))
+    grid = syn.e4m3_bits_to_fp64(np.arange(256, dtype=np.uint8))
+    grid = np.unique(grid[~np.isnan(grid)])
+    # brute force: the nearest representable value (saturation aside)
+    idx = np.abs(x[:, None] - grid[None, :]).argmin(axis=1)
+    best = np.abs(x - grid[idx])
+    assert np.all(np.abs(x - got) <= best + 1e-300)
