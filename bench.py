@@ -476,6 +476,8 @@ def run_sweep(args):
     peaks = measured_peaks()
     for name in names:
         w = syn.workload(name)
+        if args.heads is not None:
+            w = w.replace(H=min(w.H, args.heads))
         if args.fp8:
             run_sweep_fp8(args, w, dev, peaks)
             continue
@@ -736,6 +738,8 @@ def main():
     ap.add_argument("--rope-dims", type=int, default=None, help="--prep: rotated dimensions (default D/2)")
     ap.add_argument("--sweep-min-ms", type=float, default=500.0,
                     help="--sweep: lower bound on each attend timing region (more launches if needed)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="--sweep on the first H heads only (a reduced case for profiling)")
     ap.add_argument("--fp8", action="store_true",
                     help="--sweep with the 8-bit entry point (E4M3 inputs); frac against twice the bf16 peak")
     ap.add_argument("--budget-sparsity", type=float, default=None,
