@@ -3,11 +3,12 @@
 compute-sanitizer is closed on this machine, so every output buffer here sits
 inside a larger allocation whose margins hold a sentinel pattern, and the
 margins are checked after the call.  The inputs are checked to be unchanged.
-Shapes cover odd block counts (a last tile and a last four-block group with
-missing blocks), B > 1 and odd prefixes; the host-buffer entry point runs
+Shapes cover odd block counts (a last 128-row tile holding one block), B > 1
+and odd prefixes; the host-buffer entry point runs
 with uneven head chunks; the debug keep-mask export and the pooled
-workspace are guarded the same way.  Each result is also compared with the
-same call on plain buffers, so the guards cannot hide a wrong answer.
+workspace are guarded the same way, and so is the 8-bit entry point.  Each
+result is also compared with the same call on plain buffers, so the guards
+cannot hide a wrong answer.
 """
 
 import math
@@ -51,8 +52,8 @@ def _inputs(B, H, N, D, prefix, seed):
 
 
 CASES = [
-    dict(B=2, H=3, N=64 * 13, D=128, prefix=192, tau=0.8),   # M = 13: last group holds one block
-    dict(B=1, H=2, N=64 * 14, D=128, prefix=0, tau=1.0),     # M = 14: last group holds two blocks
+    dict(B=2, H=3, N=64 * 13, D=128, prefix=192, tau=0.8),   # M = 13: the last tile holds one block
+    dict(B=1, H=2, N=64 * 14, D=128, prefix=0, tau=1.0),     # M = 14: every tile holds two blocks
     dict(B=3, H=1, N=64 * 7, D=64, prefix=64, tau=0.5),      # D = 64, M = 7
     dict(B=1, H=2, N=64, D=128, prefix=0, tau=1.0),          # one block
     dict(B=1, H=2, N=64 * 9, D=128, prefix=64 * 9, tau=1.0), # all prefix
@@ -125,3 +126,21 @@ def test_host_entry_point_with_uneven_chunks_writes_only_out():
     ref = abi.forward(q, k, v, tau, L)
     torch.cuda.synchronize()
     assert torch.equal(hout, ref.cpu())
+
+
+def test_fp8_forward_writes_only_out():
+    B, H, N, D, L, tau = 2, 2, 64 * 13, 128, 192, 0.8
+    w = syn.Workload("guard8", B, H, N, D, L, (16, 24, 42), 0.8, (1.0,), 5151)
+    bits = syn.generate_e4m3(w)
+    dev = torch.device("cuda", 0)
+    q8, k8, v8 = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in bits)
+    q0, k0, v0 = q8.clone(), k8.clone(), v8.clone()
+    big, out = _guarded_bf16((B, H, N, D), dev)
+    abi.forward_fp8(q8, k8, v8, tau, L, out=out)
+    torch.cuda.synchronize()
+    assert abi.device_status() == abi.OK
+    assert _margins_intact_bf16(big, out.numel())
+    assert torch.equal(q8, q0) and torch.equal(k8, k0) and torch.equal(v8, v0)
+    ref = abi.forward_fp8(q8, k8, v8, tau, L)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
