@@ -220,6 +220,15 @@ def _oracle_rate(w, tau, budget_s, rank_seed, small, qb, kb, vb, cores, dense_bu
     return res
 
 
+def workload_config(w, tau, world: int) -> dict:
+    """The `config` object both arms print: the workload, its size against the
+    GPU's L2 (the reason no flush is needed between steps) and the replicas."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+            "prefix_len": w.prefix_len, "tau": tau, "block": 64,
+            "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2f} GB > L2 126 MB, no flush",
+            "parallelism": f"replicas x{world}"}
+
+
 # --------------------------------------------------------------------------- allocator
 
 def keep_pool_memory(device_index: int) -> bool:
@@ -420,11 +429,8 @@ def run_gpu(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded video-grid Q/K/V, no model weights)",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
-                       "prefix_len": w.prefix_len, "tau": tau, "block": 64,
-                       "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2f} GB > L2 126 MB, no flush",
-                       "parallelism": f"replicas x{world}",
-                       "mempool": "freed scratch kept by the pool" if pool_kept else "default pool"},
+            "config": workload_config(w, tau, world),
+            "mempool": "freed scratch kept by the pool" if pool_kept else "default pool",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                          "traffic": traffic, "kernel": "sol_attn_fwd_kernel<128,false>",
@@ -707,8 +713,7 @@ def run_reference(args, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded video-grid Q/K/V, no model weights)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
-                   "prefix_len": w.prefix_len, "tau": tau, "block": 64},
+        "config": workload_config(w, tau, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": o["cores"], "kind": "oracle",
                          "cpu_model": cpu_model(),
                          "sample": f"per step: routing of the first 4 heads plus ~{args.ref_step_budget:.0f} s of "

@@ -22,7 +22,8 @@ def test_reference_arm_json_line():
     assert d["metric"] == bench.METRIC
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["n_gpus"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0 and d["steps"] == 1 and d["warmup"] == 3
-    assert d["config"]["workload"] == "refine_n32768"
+    assert d["config"] == bench.workload_config(__import__("block_sparse_attention_threshold_b200.synthetic",
+                                                                  fromlist=["x"]).workload("refine_n32768"), 1.25, 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
