@@ -229,6 +229,28 @@ def workload_config(w, tau, world: int) -> dict:
             "parallelism": f"replicas x{world}"}
 
 
+# --------------------------------------------------------------------------- library comparator
+
+LIBRARY_DENSE_IMPL = "torch scaled_dot_product_attention, cuDNN backend"
+
+
+def library_dense_ms(q, k, v, timed):
+    """Dense attention on the same q, k, v through PyTorch's SDPA with its
+    cuDNN backend, timed by `timed`: context for the speedup, beside the
+    in-repo dense kernel (the pages quote their operator against a dense
+    FA-class kernel).  Returns None when that backend cannot run here."""
+    import torch
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        import torch.nn.functional as F
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            F.scaled_dot_product_attention(q, k, v)
+            torch.cuda.synchronize()
+            return timed(lambda: F.scaled_dot_product_attention(q, k, v))
+    except (RuntimeError, ImportError):
+        return None
+
+
 # --------------------------------------------------------------------------- allocator
 
 def keep_pool_memory(device_index: int) -> bool:
@@ -371,6 +393,7 @@ def run_gpu(args, rank, world, local_rank):
     pool_ms = timed(lambda: abi.pool(q, k, v, ws, stream=stream))
     attend_ms = timed(lambda: abi.attend(q, k, v, ws, tau, w.prefix_len, out=out, stream=stream))
     dense_ms = timed(lambda: abi.dense_forward(q, k, v, out=out, stream=stream))
+    lib_ms = library_dense_ms(q, k, v, timed)
     peaks = measured_peaks()
     pool_bytes = 3.0 * w.B * w.H * w.N * w.D * 2 + w.B * w.H * w.M * w.D * 12
     achieved = (kept_flops + corr_flops) / (attend_ms * 1e-3) / 1e12
@@ -443,6 +466,9 @@ def run_gpu(args, rank, world, local_rank):
                 "dense_ms": dense_ms,
                 "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                 "speedup_vs_dense": dense_ms / ms,
+                "library_dense": None if lib_ms is None else {
+                    "impl": LIBRARY_DENSE_IMPL, "ms": lib_ms,
+                    "tflops": dense_flops / (lib_ms * 1e-3) / 1e12, "speedup": lib_ms / ms},
                 "kept_frac": kept_pairs / total_pairs,
                 "exact_frac": exact_pairs / total_pairs,
                 "actual_tflops_kept": kept_flops / (attend_ms * 1e-3) / 1e12,
@@ -515,6 +541,7 @@ def run_sweep(args):
 
         pool_ms = timed(lambda: abi.pool(q, k, v, ws), args.reps)
         dense_ms = timed(lambda: abi.dense_forward(q, k, v, out=out), max(1, args.reps // 2))
+        lib_ms = library_dense_ms(q, k, v, lambda fn: timed(fn, max(1, args.reps // 2)))
         taus = [args.tau] if args.tau is not None else list(w.taus)
         budget = 0
         if args.budget_sparsity is not None:  # fixed-budget routing, skipped blocks dropped
@@ -552,6 +579,8 @@ def run_sweep(args):
                 "tensor_tflops_exact_union": exact * 4.0 * 64 * 64 * w.D / att_ms / 1e9,
                 "dense_tflops": w.dense_flops() / dense_ms / 1e9,
                 "speedup_vs_dense": dense_ms / step,
+                "library_dense_tflops": None if lib_ms is None else w.dense_flops() / lib_ms / 1e9,
+                "speedup_vs_library_dense": None if lib_ms is None else lib_ms / step,
                 "pool_gbs": (3.0 * w.B * w.H * w.N * w.D * 2 + w.B * w.H * w.M * w.D * 12) / pool_ms / 1e6,
                 "device_status": abi.device_status(),
                 "clocks": clk.summary(),

@@ -44,3 +44,16 @@ def test_cpu_baseline_times_routing_and_dense_oracle():
     per_block = o["seconds"] * o["cores"] / o["blocks"]
     want = w.B * w.H * (o["route_s_per_head"] + w.M * per_block) / o["cores"]
     assert abs(o["full_s"] - want) <= 1e-9 * want
+
+
+def test_library_dense_comparator_runs_or_reports_none():
+    # The cuDNN SDPA backend has no CPU kernel: the helper must say so with
+    # None rather than fail, and never call the timer for a backend that
+    # cannot run.
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    calls = []
+    assert bench.library_dense_ms(q, q, q, lambda fn: calls.append(fn) or 1.0) is None
+    assert calls == []
