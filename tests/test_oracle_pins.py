@@ -228,6 +228,47 @@ def test_value_shift_invariance():
     np.testing.assert_allclose(b - a, np.broadcast_to(c, a.shape), rtol=0, atol=1e-12)
 
 
+def _permute_blocks(x, order, block=64):
+    """Rows of x regrouped so that block i of the result is block order[i] of x."""
+    return np.concatenate([x[j * block:(j + 1) * block] for j in order], axis=0)
+
+
+@pytest.mark.parametrize("tau", [0.5, 1.25])
+def test_video_key_block_permutation_invariance(tau):
+    """Every output row sums over key blocks, exact or pooled, and the keep
+    rule uses the mean and std of the row's video scores: permuting the video
+    key blocks (their K and V rows together) changes no output and permutes
+    each row's keep mask with them.  A block-index slip anywhere in the
+    routing or the correction breaks this."""
+    w, q, k, v = _tiny_inputs()
+    qh, kh, vh = q[0, 0], k[0, 0], v[0, 0]
+    rng = np.random.default_rng(5)
+    order = list(range(w.P)) + list(w.P + rng.permutation(w.M - w.P))
+    kp, vp = _permute_blocks(kh, order), _permute_blocks(vh, order)
+    a = orc.solattn_blocks(qh, kh, vh, 64, w.prefix_len, tau)
+    b = orc.solattn_blocks(qh, kp, vp, 64, w.prefix_len, tau)
+    np.testing.assert_allclose(b, a, rtol=0, atol=1e-12)
+    ra = orc.route(qh, kh, 64, w.prefix_len, tau)
+    rb = orc.route(qh, kp, 64, w.prefix_len, tau)
+    assert np.array_equal(rb.keep, ra.keep[:, order])
+    assert 0 < ra.keep[w.P:, w.P:].sum() < (w.M - w.P) ** 2
+
+
+def test_query_block_permutation_moves_outputs():
+    """Query blocks do not interact: permuting the video query blocks permutes
+    their output blocks and keep rows, and nothing else."""
+    w, q, k, v = _tiny_inputs()
+    qh, kh, vh = q[0, 0], k[0, 0], v[0, 0]
+    rng = np.random.default_rng(6)
+    order = list(range(w.P)) + list(w.P + rng.permutation(w.M - w.P))
+    a = orc.solattn_blocks(qh, kh, vh, 64, w.prefix_len, 1.0)
+    b = orc.solattn_blocks(_permute_blocks(qh, order), kh, vh, 64, w.prefix_len, 1.0)
+    np.testing.assert_allclose(b, _permute_blocks(a, order), rtol=0, atol=1e-12)
+    ra = orc.route(qh, kh, 64, w.prefix_len, 1.0)
+    rb = orc.route(_permute_blocks(qh, order), kh, 64, w.prefix_len, 1.0)
+    assert np.array_equal(rb.keep, ra.keep[order, :])
+
+
 def _brute_force_head(q, k, v, block, L, tau):
     """Independent plain-loop Sol-Attn for tiny inputs (lists and math only)."""
     N, D = len(q), len(q[0])
