@@ -1,5 +1,6 @@
 """Properties of the CUDA path that hold at any size, checked at full sequence
-length (refine: N = 32768, D = 128, prefix 1024; four of its heads).
+length (refine: N = 32768, D = 128, prefix 1024; four or eight of its heads),
+where the oracle can only sample rows.
 
 Permuting the video key blocks (their K and V rows together) permutes every
 row's keep mask with them and changes no output beyond summation order: the
@@ -53,3 +54,28 @@ def test_video_key_block_permutation_full_size():
     rel = ((a - b).norm() / a.norm()).item()
     assert rel <= 2e-3, rel
     assert (a - b).abs().max().item() <= 2e-2
+
+
+def test_dense_paths_agree_with_a_library_kernel_on_every_row():
+    """A cross-check, not parity (parity is against the CPU oracle, which can
+    only sample rows at this length): on every row of refine's full length,
+    the in-repo dense kernel and Sol-Attn at tau = -inf (which keeps every
+    block) agree with cuDNN's dense attention through PyTorch's SDPA, up to
+    the rounding of two fp32-accumulating bf16 kernels."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    import torch.nn.functional as F
+    w = syn.workload("refine_n32768").replace(H=8)
+    q, k, v = parity.to_device(*syn.generate_bf16(w))
+    try:
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            ref = F.scaled_dot_product_attention(q, k, v).float()
+    except RuntimeError as e:  # the backend is not built for this device
+        pytest.skip(f"cuDNN SDPA unavailable: {e}")
+    dense = abi.dense_forward(q, k, v)
+    sol = abi.forward(q, k, v, float("-inf"), w.prefix_len)
+    torch.cuda.synchronize()
+    assert abi.device_status() == abi.OK
+    for out in (dense, sol):
+        d = out.float() - ref
+        assert (d.norm() / ref.norm()).item() <= 5e-3
+        assert d.abs().max().item() <= 2e-2
