@@ -1,6 +1,6 @@
 """Properties of the CUDA path that hold at any size, checked at full sequence
-length (refine: N = 32768, D = 128, prefix 1024; four or eight of its heads),
-where the oracle can only sample rows: a block permutation, agreement of the
+length (refine, N = 32768, four or eight of its heads; the 131072-token sweep
+workload, one head), where the oracle can only sample rows: a block permutation, agreement of the
 dense paths with a library dense kernel, and every output row against the
 definition written out in fp32 PyTorch.
 
@@ -83,7 +83,8 @@ def test_dense_paths_agree_with_a_library_kernel_on_every_row():
         assert d.abs().max().item() <= 2e-2
 
 
-def test_every_row_matches_an_fp32_reference_at_full_length():
+@pytest.mark.parametrize("name,heads,tau", [("refine_n32768", 4, 1.25), ("sweep_n131072", 1, 1.25)])
+def test_every_row_matches_an_fp32_reference_at_full_length(name, heads, tau):
     """Every output row at refine's full length against the Sol-Attn
     definition written out here in fp32 PyTorch (library matmuls and softmax,
     no TF32).  The output is compared under the kernel's own keep mask (the
@@ -92,8 +93,7 @@ def test_every_row_matches_an_fp32_reference_at_full_length():
     the video key blocks, keep iff score >= mean + tau * std).  Parity with
     the fp64 oracle stays the sampled test; this covers the rows it skips."""
     torch.backends.cuda.matmul.allow_tf32 = False
-    w = syn.workload("refine_n32768").replace(H=4)
-    tau = 1.25
+    w = syn.workload(name).replace(H=heads)
     q, k, v = parity.to_device(*syn.generate_bf16(w))
     out, keep, _, _ = parity.run_sol(w, tau, q, k, v)
     keep = torch.from_numpy(keep).to(q.device)
