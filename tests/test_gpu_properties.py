@@ -2,7 +2,7 @@
 length (refine, N = 32768, four or eight of its heads; the 131072-token sweep
 workload, one head), where the oracle can only sample rows: a block permutation, agreement of the
 dense paths with a library dense kernel, and every output row against the
-definition written out in fp32 PyTorch.
+definition written out in fp32 PyTorch (bf16 and E4M3 entry points).
 
 Permuting the video key blocks (their K and V rows together) permutes every
 row's keep mask with them and changes no output beyond summation order: the
@@ -83,23 +83,14 @@ def test_dense_paths_agree_with_a_library_kernel_on_every_row():
         assert d.abs().max().item() <= 2e-2
 
 
-@pytest.mark.parametrize("name,heads,tau", [("refine_n32768", 4, 1.25), ("sweep_n131072", 1, 1.25)])
-def test_every_row_matches_an_fp32_reference_at_full_length(name, heads, tau):
-    """Every output row at refine's full length against the Sol-Attn
-    definition written out here in fp32 PyTorch (library matmuls and softmax,
-    no TF32).  The output is compared under the kernel's own keep mask (the
-    debug export), so threshold ties cannot blur it; the mask itself is
-    checked against fp32 routing done here (pooled means, population std over
-    the video key blocks, keep iff score >= mean + tau * std).  Parity with
-    the fp64 oracle stays the sampled test; this covers the rows it skips."""
+def _check_against_fp32_reference(w, tau, qf, kf, vf, out, keep, rel_bar, abs_bar):
+    """Routing and output of one run against the Sol-Attn definition in fp32
+    PyTorch: the mask against fp32 routing done here, every output row under
+    the kernel's own mask."""
     torch.backends.cuda.matmul.allow_tf32 = False
-    w = syn.workload(name).replace(H=heads)
-    q, k, v = parity.to_device(*syn.generate_bf16(w))
-    out, keep, _, _ = parity.run_sol(w, tau, q, k, v)
-    keep = torch.from_numpy(keep).to(q.device)
+    keep = torch.from_numpy(keep).to(qf.device)
     B, H, N, D, M, P = w.B, w.H, w.N, w.D, w.M, w.P
     scale = D ** -0.5
-    qf, kf, vf = q.float(), k.float(), v.float()
     qbar, kbar, vbar = (x.view(B, H, M, 64, D).mean(3) for x in (qf, kf, vf))
     # routing in fp32
     s = scale * qbar[:, :, P:] @ kbar[:, :, P:].transpose(-1, -2)       # [B, H, M-P, M-P]
@@ -111,7 +102,7 @@ def test_every_row_matches_an_fp32_reference_at_full_length(name, heads, tau):
     assert keep[:, :, :P].all() and keep[:, :, :, :P].all()
     # output under the kernel's mask, eight query blocks at a time
     worst_rel, worst_abs = 0.0, 0.0
-    ln_c = torch.log(torch.tensor(64.0, device=q.device))
+    ln_c = torch.log(torch.tensor(64.0, device=qf.device))
     for b in range(B):
         for h in range(H):
             num = den = 0.0
@@ -130,5 +121,41 @@ def test_every_row_matches_an_fp32_reference_at_full_length(name, heads, tau):
                 den += ref.square().sum().item()
                 worst_abs = max(worst_abs, d.abs().max().item())
             worst_rel = max(worst_rel, (num / den) ** 0.5)
-    assert worst_rel <= parity.REL_L2, worst_rel
-    assert worst_abs <= parity.MAX_ABS, worst_abs
+    assert worst_rel <= rel_bar, worst_rel
+    assert worst_abs <= abs_bar, worst_abs
+
+
+@pytest.mark.parametrize("name,heads,tau", [("refine_n32768", 4, 1.25), ("sweep_n131072", 1, 1.25)])
+def test_every_row_matches_an_fp32_reference_at_full_length(name, heads, tau):
+    """Every output row at full length against the Sol-Attn definition
+    written out here in fp32 PyTorch (library matmuls and softmax, no TF32).
+    The output is compared under the kernel's own keep mask (the debug
+    export), so threshold ties cannot blur it; the mask itself is checked
+    against fp32 routing done here (pooled means, population std over the
+    video key blocks, keep iff score >= mean + tau * std).  Parity with the
+    fp64 oracle stays the sampled test; this covers the rows it skips."""
+    w = syn.workload(name).replace(H=heads)
+    q, k, v = parity.to_device(*syn.generate_bf16(w))
+    out, keep, _, _ = parity.run_sol(w, tau, q, k, v)
+    _check_against_fp32_reference(w, tau, q.float(), k.float(), v.float(), out, keep,
+                                  parity.REL_L2, parity.MAX_ABS)
+
+
+def test_every_row_of_the_8bit_path_matches_an_fp32_reference():
+    """The E4M3 entry point, refine at full length (four heads, scales 0.5,
+    2 and 0.25), against the same fp32 reference on the decoded inputs times
+    their scales, at the 8-bit bar (rel-L2 <= 5e-2, max-abs <= 1e-1)."""
+    w = syn.workload("refine_n32768").replace(H=4)
+    tau, scales = 1.25, (0.5, 2.0, 0.25)
+    dev = torch.device("cuda", 0)
+    q8, k8, v8 = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in syn.generate_e4m3(w, scales))
+    M = w.M
+    mask = torch.zeros(w.B * w.H * M * abi.mask_words(M), dtype=torch.int32, device=dev)
+    opts = abi.Opts()
+    opts.debug_mask = mask.data_ptr()
+    out = abi.forward_fp8(q8, k8, v8, tau, w.prefix_len, *scales, opts=opts)
+    torch.cuda.synchronize()
+    assert abi.device_status() == abi.OK
+    keep = abi.unpack_mask(mask.cpu().numpy().view(np.uint32).reshape(w.B, w.H, M, -1), M)
+    qf, kf, vf = (x.view(torch.float8_e4m3fn).float() * sc for x, sc in zip((q8, k8, v8), scales))
+    _check_against_fp32_reference(w, tau, qf, kf, vf, out, keep, 5e-2, 1e-1)
