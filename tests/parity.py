@@ -165,3 +165,36 @@ def assert_parity(m, rel_l2=REL_L2, max_abs=MAX_ABS):
         assert m["mask_agree"] >= MASK_AGREE, m
         assert m["worst_band"] <= MASK_BAND, m
         assert m["hard_mismatch"] == 0, m
+
+
+# ----------------------------------------------------------------------------- fp32 reference
+
+def fp32_route(w, tau, qf, kf):
+    """Keep bits of the video part ([B, H, M-P, M-P]) from the definition in
+    fp32 PyTorch: pooled means, population std over the video key blocks,
+    keep iff score >= mean + tau * std.  qf, kf: float32 [B, H, N, D] on any
+    device.  A cross-check for full-length runs; the oracle stays the
+    authority (tests/test_parity_harness.py pins this to it)."""
+    B, H, N, D, M, P = w.B, w.H, w.N, w.D, w.M, w.P
+    qbar, kbar = (x.view(B, H, M, 64, D).mean(3) for x in (qf, kf))
+    s = (D ** -0.5) * qbar[:, :, P:] @ kbar[:, :, P:].transpose(-1, -2)
+    mu = s.mean(-1, keepdim=True)
+    sd = s.std(-1, unbiased=False, keepdim=True)
+    return s >= mu + tau * sd
+
+
+def fp32_rows(w, qf, kf, vf, keep, b, h, i0, i1):
+    """Output rows of query blocks [i0, i1) of head (b, h) under the keep
+    mask `keep` (bool [B, H, M, M], same device): exact logits over kept
+    blocks, pooled logits + ln 64 with the pooled value over skipped ones, one
+    softmax, in fp32 PyTorch."""
+    import torch
+    N, D, M = w.N, w.D, w.M
+    scale = D ** -0.5
+    kbar, vbar = (x[b, h].view(M, 64, D).mean(1) for x in (kf, vf))
+    qc = qf[b, h, i0 * 64:i1 * 64]
+    kb = keep[b, h, i0:i1].repeat_interleave(64, dim=0)                 # [rows, M]
+    ex = (scale * qc @ kf[b, h].T).masked_fill(~kb.repeat_interleave(64, dim=1), float("-inf"))
+    po = (scale * qc @ kbar.T + math.log(64.0)).masked_fill(kb, float("-inf"))
+    p = torch.softmax(torch.cat([ex, po], dim=1), dim=1)
+    return p[:, :N] @ vf[b, h] + p[:, N:] @ vbar

@@ -85,38 +85,24 @@ def test_dense_paths_agree_with_a_library_kernel_on_every_row():
 
 def _check_against_fp32_reference(w, tau, qf, kf, vf, out, keep, rel_bar, abs_bar):
     """Routing and output of one run against the Sol-Attn definition in fp32
-    PyTorch: the mask against fp32 routing done here, every output row under
-    the kernel's own mask."""
+    PyTorch (parity.fp32_route / fp32_rows, themselves pinned to the oracle
+    on the CPU): the mask against fp32 routing, every output row under the
+    kernel's own mask."""
     torch.backends.cuda.matmul.allow_tf32 = False
     keep = torch.from_numpy(keep).to(qf.device)
-    B, H, N, D, M, P = w.B, w.H, w.N, w.D, w.M, w.P
-    scale = D ** -0.5
-    qbar, kbar, vbar = (x.view(B, H, M, 64, D).mean(3) for x in (qf, kf, vf))
-    # routing in fp32
-    s = scale * qbar[:, :, P:] @ kbar[:, :, P:].transpose(-1, -2)       # [B, H, M-P, M-P]
-    mu = s.mean(-1, keepdim=True)
-    sd = s.std(-1, unbiased=False, keepdim=True)
-    mine = s >= mu + tau * sd
+    P = w.P
+    mine = parity.fp32_route(w, tau, qf, kf)
     agree = (mine == keep[:, :, P:, P:]).float().mean().item()
     assert agree >= 0.999, agree
     assert keep[:, :, :P].all() and keep[:, :, :, :P].all()
-    # output under the kernel's mask, eight query blocks at a time
     worst_rel, worst_abs = 0.0, 0.0
-    ln_c = torch.log(torch.tensor(64.0, device=qf.device))
-    for b in range(B):
-        for h in range(H):
+    for b in range(w.B):
+        for h in range(w.H):
             num = den = 0.0
-            for i0 in range(0, M, 8):
-                i1 = min(M, i0 + 8)
-                rows = slice(i0 * 64, i1 * 64)
-                qc = qf[b, h, rows]
-                kb = keep[b, h, i0:i1].repeat_interleave(64, dim=0)       # [rows, M]
-                ex = scale * qc @ kf[b, h].T                              # [rows, N]
-                ex = ex.masked_fill(~kb.repeat_interleave(64, dim=1), float("-inf"))
-                po = (scale * qc @ kbar[b, h].T + ln_c).masked_fill(kb, float("-inf"))
-                p = torch.softmax(torch.cat([ex, po], dim=1), dim=1)
-                ref = p[:, :N] @ vf[b, h] + p[:, N:] @ vbar[b, h]
-                d = out[b, h, rows].float() - ref
+            for i0 in range(0, w.M, 8):               # eight query blocks at a time
+                i1 = min(w.M, i0 + 8)
+                ref = parity.fp32_rows(w, qf, kf, vf, keep, b, h, i0, i1)
+                d = out[b, h, i0 * 64:i1 * 64].float() - ref
                 num += d.square().sum().item()
                 den += ref.square().sum().item()
                 worst_abs = max(worst_abs, d.abs().max().item())

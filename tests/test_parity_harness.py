@@ -73,3 +73,23 @@ def test_harness_measures_routed_mismatch_against_sigma():
     m = parity.oracle_compare(w, 1.0, *bits, out, bad, workers=2)
     assert m["hard_mismatch"] == 0 and m["mask_mismatch"] == 1
     assert m["worst_band"] == pytest.approx(abs(r.score[i, j] - r.thr[i]) / r.sigma[i])
+
+
+@pytest.mark.parametrize("tau", [0.5, 1.0, 1.5])
+def test_fp32_reference_matches_the_oracle(tau):
+    """The fp32 PyTorch reference that the full-length GPU checks use, pinned
+    to the oracle on the tiny workload: the same keep mask and the same rows."""
+    import torch
+    w = syn.workload("tiny_n1024")
+    q, k, v = (syn.bf16_bits_to_fp64(a) for a in syn.generate_bf16(w))
+    qf, kf, vf = (torch.from_numpy(x).float() for x in (q, k, v))
+    mine = parity.fp32_route(w, tau, qf, kf).numpy()
+    keep = np.stack([np.stack([orc.route(q[b, h], k[b, h], 64, w.prefix_len, tau).keep
+                               for h in range(w.H)]) for b in range(w.B)])
+    assert np.array_equal(mine, keep[:, :, w.P:, w.P:])
+    ref = orc.solattn(q, k, v, 64, w.prefix_len, tau)
+    kt = torch.from_numpy(keep)
+    for b in range(w.B):
+        for h in range(w.H):
+            rows = parity.fp32_rows(w, qf, kf, vf, kt, b, h, 0, w.M).double().numpy()
+            np.testing.assert_allclose(rows, ref[b, h], rtol=0, atol=2e-5)
